@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 decode GEMV: microseconds per linear and achieved
+HBM bandwidth at M = 1 on the 8192 x 28672 (N x K) Llama-70B-shaped linear
+(asymmetric uint4, G = 128, fp16 scale and zero), one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one decode linear y = x dequant(Wq)^T through wq_gemv_w4a16 with the
+quantized weights resident in HBM.  Quantization and relayout are the offline
+part of the path (done once per model); they run and are timed in the same
+process and reported under "offline".  The timed region replays CUDA graphs of
+back-to-back GEMV launches that cycle through several copies of the packed
+weight (more bytes than L2 holds), bracketed by CUDA events on the launching
+stream, with a barrier and a device synchronize on both sides; with N > 1
+every rank runs its own replica and the slowest rank's time counts.
+
+--impl reference times the CPU oracle (the plain C restatement of the method)
+on the host cores instead, one output row per step, scaled to a full linear.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime as dt
+import hashlib
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 G128 GEMV µs/linear and achieved HBM TB/s vs B200 peak at M=1"
+UNIT = "us/linear"
+WORKLOAD_CID, WORKLOAD_LIN = 3, 3          # Llama-70B-shaped linear, N=8192, K=28672
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
+# reported only while the sources are unchanged.
+NCU_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None}
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the offline and other-M legs")
+    return ap.parse_args()
+
+
+def algorithmic_bytes(M: int, N: int, K: int, sym: bool) -> int:
+    """Bytes the method must move for one linear: packed codes, fp16 scales,
+    fp16 zeros (asymmetric), bf16 x and fp32 y."""
+    return N * K // 2 + 2 * N * K // 128 + (0 if sym else 2 * N * K // 128) + 2 * M * K + 4 * M * N
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("wq_gemv.cu", "wq_common.cuh"):
+        with open(os.path.join(ROOT, "post_weight_quantization_wq_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (copy bandwidth, measured)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier measurement on this pool)"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons, kept only while
+    the timed region runs (by wall-clock timestamp)."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark_begin(self):
+        self.t0 = dt.datetime.now()
+
+    def mark_end(self):
+        self.t1 = dt.datetime.now()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for rec in csv.reader(io.StringIO(out)):
+            if len(rec) < 9:
+                continue
+            rec = [r.strip() for r in rec]
+            try:
+                ts = dt.datetime.strptime(rec[0], "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                continue
+            if self.t0 and self.t1 and not (self.t0 <= ts <= self.t1):
+                continue
+            rows.append(rec)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for rec in rows for n, v in zip(names, rec[5:9]) if v == "Active"})
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(a, rank: int, world: int, local_rank: int):
+    import numpy as np
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    from post_weight_quantization_wq_b200 import _binding as abi
+    from post_weight_quantization_wq_b200 import inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    wl = inputs.WORKLOADS[WORKLOAD_CID]
+    lin = wl.linears[WORKLOAD_LIN]
+    N, K, M, sym = lin.N, lin.K, 1, wl.sym
+
+    W = inputs.workload_weight(WORKLOAD_CID, WORKLOAD_LIN)
+    x = inputs.workload_activations(WORKLOAD_CID, WORKLOAD_LIN, M)
+    Wt = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+    xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    extras = {}
+    with torch.cuda.stream(stream):
+        qw = wq.quantize(Wt, symmetric=sym, stream=stream)
+        if not a.no_extras:
+            extras["offline"] = time_offline(Wt, qw, stream, N, K, sym)
+    torch.cuda.synchronize(dev)
+    del Wt
+
+    # L2 hygiene: cycle through copies of the packed weight, more bytes than L2.
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    wbytes = qw.packed.numel()
+    ncopies = max(3, math.ceil(3 * l2 / wbytes))
+    copies = [qw.packed] + [qw.packed.clone() for _ in range(ncopies - 1)]
+    ws_bytes = abi.wq_workspace_bytes(M, N, K)
+    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+
+    def launch(i, s):
+        st = abi.wq_gemv_w4a16(xt, None, copies[i % ncopies], M, N, K, 128, sym, 1, y, ws,
+                               ws_bytes, s)
+        if st != 0:
+            raise wq.WqError(st, "wq_gemv_w4a16")
+
+    chunk = 100 * ncopies
+    graphs = build_graphs(launch, stream, a.steps, chunk, dev)
+
+    # warm-up (untimed)
+    with torch.cuda.stream(stream):
+        for i in range(a.warmup):
+            launch(i, stream)
+    torch.cuda.synchronize(dev)
+    if abi.wq_last_device_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    sampler = None
+    if rank == 0:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):          # graph replays go to the current stream
+        e0.record(stream)
+        for g in graphs:
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_end()
+    barrier(world)
+    elapsed_ms = e0.elapsed_time(e1)
+    clocks = sampler.stop() if sampler else None
+    st = abi.wq_last_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {abi.status_string(st)}")
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+
+    # correctness spot check of the timed configuration (cheap): y vs a second
+    # launch on another copy must be bit-identical (fixed reduction order)
+    y_timed = y.clone()
+    with torch.cuda.stream(stream):
+        launch(1, stream)
+    torch.cuda.synchronize(dev)
+    deterministic = bool(torch.equal(y, y_timed))
+
+    e2e = run_e2e(a, qw, copies, ncopies, x, M, N, K, sym, dev, stream, ws, ws_bytes, world)
+
+    if not a.no_extras:
+        extras["other_m"] = time_other_m(qw, copies, ncopies, N, K, sym, dev, stream)
+
+    bytes_per = algorithmic_bytes(M, N, K, sym)
+    us_per_launch = elapsed_ms * 1e3 / a.steps
+    achieved_gbs = bytes_per / (us_per_launch * 1e-6) / 1e9
+    peak, peak_src = measured_peaks()
+    traffic = None
+    if NCU_TRAFFIC["sources_sha256"] == kernel_sources_sha():
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    value = elapsed_ms * 1e3 / (a.steps * world)
+
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": elapsed_ms / a.steps,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "llama70b_down_8192x28672_asym_g128_m1", "N": N, "K": K, "M": M,
+                   "group_size": 128, "symmetric": sym, "weights": "N(0,0.015) bf16, seeded PCG64",
+                   "l2": f"rotating {ncopies} packed-weight copies "
+                         f"({ncopies * wbytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
+                   "timing": "CUDA graphs of back-to-back GEMV launches, CUDA events",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "hbm_tbs": round(achieved_gbs / 1e3, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved_gbs / peak, 4), "traffic": traffic,
+                     "bytes_per_launch": bytes_per, "peak_source": peak_src,
+                     "frac_of_nominal_8tbs": round(achieved_gbs / 8000.0, 4)},
+        "gpu_launches": a.steps,
+        "deterministic": deterministic,
+        "e2e": e2e,
+        "clocks": clocks,
+    }
+    line.update(extras)
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(W, x, N, K, sym)
+    return line
+
+
+def build_graphs(launch, stream, steps, chunk, dev):
+    import torch
+    graphs = []
+    # make sure the first launch (one-time set-up) happens outside capture
+    with torch.cuda.stream(stream):
+        launch(0, stream)
+    torch.cuda.synchronize(dev)
+    sizes = [chunk] * (steps // chunk) + ([steps % chunk] if steps % chunk else [])
+    cache = {}
+    for n in sizes:
+        if n not in cache:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    launch(i, stream)
+            cache[n] = g
+        graphs.append(cache[n])
+    return graphs
+
+
+def time_offline(Wt, qw, stream, N, K, sym):
+    """Quantize + relayout timings for the same weight (events, 5 reps each;
+    the 470 MB bf16 input exceeds L2)."""
+    import torch
+    from post_weight_quantization_wq_b200 import _binding as abi
+    reps = 5
+    d_status = torch.zeros(4, dtype=torch.int32, device=Wt.device)
+    res = {}
+    for name, fn in (
+        ("quantize_rtn", lambda: abi.wq_quantize_rtn(Wt, None, N, K, 128, sym, qw.qweight,
+                                                     qw.scales, qw.zeros, d_status, stream)),
+        ("pack_layout", lambda: abi.wq_pack_layout(qw.qweight, qw.scales, qw.zeros, N, K, 128,
+                                                   sym, 1, qw.packed, qw.packed.numel(),
+                                                   stream))):
+        fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            st = fn()
+            assert st == 0
+        e1.record(stream)
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        if name == "quantize_rtn":
+            nbytes = 2 * N * K + N * K // 2 + 2 * N * K // 128 * (1 if sym else 2)
+        else:
+            nbytes = 2 * (N * K // 2 + 2 * N * K // 128 * (1 if sym else 2))
+        res[name] = {"us": round(us, 2), "bytes": nbytes,
+                     "gbs": round(nbytes / (us * 1e-6) / 1e9, 1)}
+    return res
+
+
+def time_other_m(qw, copies, ncopies, N, K, sym, dev, stream):
+    """GEMV at M = 2, 4, 8 on the same weight (2000 launches each, graphs)."""
+    import numpy as np
+    import torch
+    from post_weight_quantization_wq_b200 import _binding as abi
+    from post_weight_quantization_wq_b200 import inputs
+    out = {}
+    for M in (2, 4, 8):
+        x = inputs.workload_activations(WORKLOAD_CID, WORKLOAD_LIN, M)
+        xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        ws_bytes = abi.wq_workspace_bytes(M, N, K)
+        ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+        def launch(i, s):
+            st = abi.wq_gemv_w4a16(xt, None, copies[i % ncopies], M, N, K, 128, sym, 1, y, ws,
+                                   ws_bytes, s)
+            assert st == 0
+
+        steps = 2000
+        graphs = build_graphs(launch, stream, steps, 100 * ncopies, dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for g in graphs[:2]:
+                g.replay()
+            e0.record(stream)
+            for g in graphs:
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / steps
+        b = algorithmic_bytes(M, N, K, sym)
+        out[str(M)] = {"us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1)}
+    return out
+
+
+def run_e2e(a, qw, copies, ncopies, x, M, N, K, sym, dev, stream, ws, ws_bytes, world):
+    """Each step: pinned host x -> device, GEMV through the public binding,
+    device y -> pinned host; timed with events around all steps."""
+    import numpy as np
+    import torch
+    from post_weight_quantization_wq_b200 import _binding as abi
+    steps = min(a.steps, 20000)
+    x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x_host, device=dev)
+    y_dev = torch.empty((M, N), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(min(a.warmup, 50)):
+            x_dev.copy_(x_host, non_blocking=True)
+            abi.wq_gemv_w4a16(x_dev, None, copies[i % ncopies], M, N, K, 128, sym, 1, y_dev,
+                              ws, ws_bytes, stream)
+            y_host.copy_(y_dev, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(steps):
+            x_dev.copy_(x_host, non_blocking=True)
+            st = abi.wq_gemv_w4a16(x_dev, None, copies[i % ncopies], M, N, K, 128, sym, 1,
+                                   y_dev, ws, ws_bytes, stream)
+            if st != 0:
+                raise RuntimeError(abi.status_string(st))
+            y_host.copy_(y_dev, non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    barrier(world)
+    return {"value": round(ms * 1e3 / (steps * world), 4), "unit": UNIT,
+            "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": y_host.numel() * 4,
+            "steps": steps, "path": "pinned host x -> device, wq_gemv_w4a16 via ctypes, "
+                                    "device y -> pinned host, per step from Python"}
+
+
+def cpu_baseline(W, x, N, K, sym, target_s: float = 10.0):
+    """The CPU oracle (single-threaded C, fp64) on a bounded sample of output
+    rows of the same linear, scaled to one full linear."""
+    import numpy as np
+    import oracle
+    rows0 = 64
+    q, s, z, _ = oracle.quantize_bf16(W[:rows0], None, sym=sym)
+    P = oracle.pack_u4(q, sym)
+    t = time.perf_counter()
+    oracle.linear(x, P, s, z, K, sym=sym)
+    per_row = (time.perf_counter() - t) / rows0
+    R = int(min(N, max(rows0, target_s / max(per_row, 1e-9))))
+    q, s, z, _ = oracle.quantize_bf16(W[:R], None, sym=sym)
+    P = oracle.pack_u4(q, sym)
+    del q
+    t = time.perf_counter()
+    oracle.linear(x, P, s, z, K, sym=sym)
+    el = time.perf_counter() - t
+    return {"value": round(el / R * N * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{R} of {N} output rows of the 8192x28672 linear at M=1 (fp64 C oracle, "
+                      f"dequantize + dot per row), {el:.1f} s, scaled to the full linear",
+            "host_cpu": _cpu_model(), "host_cores_available": os.cpu_count()}
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(a, rank: int, world: int):
+    """The CPU oracle as the reference arm: each step computes one output row
+    of the 8192 x 28672 linear at M = 1 (dequantize + fp64 dot), cycling over
+    the rows of a sampled block; value = mean step time x N."""
+    import numpy as np
+    import oracle
+    from post_weight_quantization_wq_b200 import inputs
+    wl = inputs.WORKLOADS[WORKLOAD_CID]
+    lin = wl.linears[WORKLOAD_LIN]
+    N, K, sym = lin.N, lin.K, wl.sym
+    W = inputs.workload_weight(WORKLOAD_CID, WORKLOAD_LIN)
+    x = inputs.workload_activations(WORKLOAD_CID, WORKLOAD_LIN, 1)
+    R = 256
+    q, s, z, _ = oracle.quantize_bf16(W[:R], None, sym=sym)
+    P = oracle.pack_u4(q, sym)
+    del W, q
+    rows = [np.array([i], np.int64) for i in range(R)]
+    for i in range(a.warmup):
+        oracle.linear(x, P, s, z, K, sym=sym, rows=rows[i % R])
+    # bound the run: at most ~120 s of steps
+    t0 = time.perf_counter()
+    oracle.linear(x, P, s, z, K, sym=sym, rows=rows[0])
+    per = time.perf_counter() - t0
+    steps = min(a.steps, max(1, int(120.0 / max(per, 1e-9))))
+    t0 = time.perf_counter()
+    for i in range(steps):
+        oracle.linear(x, P, s, z, K, sym=sym, rows=rows[i % R])
+    el = time.perf_counter() - t0
+    value = el / steps * N * 1e6
+    sample = (f"{steps} steps of one output row each (rows 0..{R - 1} of the 8192x28672 linear, "
+              f"M=1, fp64 C oracle), mean step time x {N} rows")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+        "n_gpus": world, "steps": steps, "warmup": a.warmup, "ms_per_step": el / steps * 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "llama70b_down_8192x28672_asym_g128_m1", "N": N, "K": K, "M": 1,
+                   "group_size": 128, "symmetric": sym},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+# ------------------------------------------------------------------ distributed
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+
+
+def max_over_ranks(v, world, dev):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    a = _args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(a, rank, world)), flush=True)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=dt.timedelta(seconds=300),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(a, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * wq.h -- C ABI of the B200 (sm_100a) library for 4-bit per-group weight
+ * quantization and the W4A16 decode linear.
+ *
+ * The problem, as the quantization pages state it:
+ *   - a linear layer computes Y = X W^T with W: [out_features, in_features]
+ *     = [N][K], and per-group quantization cuts each row of W into groups of
+ *     G consecutive input channels ("大模型量化全景解析", section
+ *     粒度和矩阵维度的关系);
+ *   - weight-only quantization stores Q(W) plus scale/zero metadata and
+ *     computes Y_hat = X dequant(Q(W))^T (same page, section
+ *     公式补课：从一层 Linear 看量化到底改了什么); the 4-bit weights are
+ *     dequantized inside the matmul kernel and multiplied with 16-bit
+ *     activations ("3.6 量化(Quantization)", section 仅权重 vs 权重 + 激活);
+ *   - the uniform quantizer is q = clamp(round(w/s) + z, qmin, qmax),
+ *     w_hat = s (q - z); symmetric: z = 0, s = max|w| / 7, q in [-7, 7];
+ *     asymmetric: s = (max - min) / 15, z = round(-min / s), q in [0, 15]
+ *     ("3.6 量化(Quantization)", section 对称与非对称量化; "后训练量化（PTQ,
+ *     Post-Training Quantization）", section 基础量化公式; "量化" compendium,
+ *     section 量化方程);
+ *   - the AWQ variant scales input channels before quantizing, W' = W diag(s),
+ *     and undoes it on the activations, Y = X diag(s)^-1 quant(W')^T
+ *     ("后训练量化（PTQ, Post-Training Quantization）", section AWQ, steps 3-5;
+ *     "3.6 量化(Quantization)", section AWQ).
+ *
+ * Conventions shared by every call:
+ *   - every pointer argument is a DEVICE pointer owned by the caller; the
+ *     library allocates, frees and synchronizes nothing (except
+ *     wq_last_device_status, which synchronizes the given stream);
+ *   - every compute call only enqueues work on `stream` and returns at once;
+ *   - arguments are validated synchronously, before anything is enqueued; a
+ *     call that returns an error has enqueued nothing;
+ *   - all matrices are dense and row-major; N, K are the output / input
+ *     dimensions of the linear, M the number of activation rows;
+ *   - pointers must be 16-byte aligned (WQ_ERR_MISALIGNED), except d_status
+ *     (4-byte aligned);
+ *   - group_size must be WQ_GROUP_SIZE and K a multiple of it
+ *     (WQ_ERR_UNSUPPORTED_SHAPE); N and K are at most WQ_MAX_DIM;
+ *   - the functions are thread-safe; the only state the library keeps is one
+ *     device error word per GPU, read by wq_last_device_status.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA stream type (identical to cudaStream_t / CUstream); NULL is the
+ * legacy default stream. */
+typedef struct CUstream_st* wq_stream_t;
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_INVALID_ARG = 1,        /* NULL where a buffer is required, bad flag, buffer too small */
+    WQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 128 != 0, group_size != 128, M out of range, dims too large */
+    WQ_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+    WQ_ERR_WORKSPACE_TOO_SMALL = 4,
+    WQ_ERR_NONFINITE = 5,          /* reported through d_status only (see wq_quantize_rtn) */
+    WQ_ERR_TIMEOUT = 6,            /* a bounded wait inside a kernel gave up */
+    WQ_ERR_CUDA = 7                /* the CUDA runtime reported an error (launch or stream) */
+} wq_status;
+
+#define WQ_GROUP_SIZE 128
+#define WQ_MAX_DIM (1 << 20)
+#define WQ_LAYOUT_TILED 1
+
+/* Human-readable name of a status code; never NULL. */
+const char* wq_status_string(int status);
+
+/* ABI version of this header (bumped on any incompatible change). */
+int wq_abi_version(void);
+#define WQ_ABI_VERSION 1
+
+/*
+ * wq_quantize_rtn -- per-group round-to-nearest 4-bit quantization plus
+ * canonical packing ("3.6 量化(Quantization)", sections 对称与非对称量化 and
+ * 粒度; "后训练量化（PTQ, Post-Training Quantization）", section 基础量化公式).
+ *
+ *   W          bf16 [N][K]: the weight, row n = output channel.
+ *   awq_scale  fp32 [K] or NULL: AWQ per-input-channel scale s; when given,
+ *              w' = fp32(W[n][k]) * s[k] (one rounded fp32 product) is
+ *              quantized instead of W.
+ *   group_size must be 128; groups are 128 consecutive k of one row.
+ *   symmetric  1: z = 0, s = max|w|/7, q = clamp(rne(w/s16), -7, 7), stored
+ *              as q + 8 (1..15);  0: s = (max-min)/15, z = rne(-min/s16),
+ *              q = clamp(rne(w/s16) + z, 0, 15), stored as q.
+ *   qweight    uint32 [N][K/8] out: element k = 8j + i of row n is nibble i
+ *              (bits [4i, 4i+4)) of qweight[n][j].
+ *   scales     fp16 [N][K/128] out: s16 = fp16_rne(max(range, 1e-8) / qden),
+ *              range and division in fp32; an s16 that rounds to 0 becomes
+ *              2^-24.  The codes are computed with this stored s16.
+ *   zeros      fp16 [N][K/128] out when symmetric == 0 (must be NULL when
+ *              symmetric == 1): z16 = fp16(rne(-min / s16)), an integer
+ *              (stored as +0 when zero); the codes use this stored z16.
+ *   d_status   int32 on device, or NULL: set to the number of non-finite
+ *              groups (a NaN/Inf input after the AWQ product, or an fp16
+ *              scale or zero that overflows).  Such a group is written as
+ *              nibbles 0 with scale (and zero) 0x7E00 (fp16 NaN), so a linear
+ *              that reads it yields NaN.  0 means every group is finite.
+ *   Rounding is round-half-to-even throughout; divisions are IEEE fp32.
+ *   Returns WQ_OK once enqueued.
+ */
+wq_status wq_quantize_rtn(const void* W, const float* awq_scale, int N, int K, int group_size,
+                          int symmetric, uint32_t* qweight, void* scales, void* zeros,
+                          int* d_status, wq_stream_t stream);
+
+/*
+ * wq_packed_bytes -- size in bytes of the kernel layout `layout` for an
+ * N x K weight; 0 if the arguments are invalid.
+ *
+ * Layout WQ_LAYOUT_TILED: the weight is cut into tiles of 128 rows x one
+ * K-slab of 4 groups (512 inputs; the last slab may hold fewer groups).
+ * Tiles are stored slab by slab and, within a slab, row-tile by row-tile;
+ * every full tile has the same size, so tile (s, b) starts at
+ * s * NB * full_tile + b * tile_bytes(s) with NB = ceil(N/128).  A tile holds
+ * first the codes (row r: its canonical qweight words for the slab's gs
+ * groups, gs*64 bytes at offset r*gs*64), then the metadata (entry (r, g) at
+ * offset 128*gs*64 + (r*gs + g) * mb): mb = 2, the fp16 scale, when
+ * symmetric; mb = 4, the fp16 scale in the low and the fp16 zero in the high
+ * half of a little-endian uint32, when asymmetric.  Rows past N are zero.
+ */
+size_t wq_packed_bytes(int N, int K, int group_size, int symmetric, int layout);
+
+/*
+ * wq_pack_layout -- permute the canonical (qweight, scales, zeros) produced
+ * by wq_quantize_rtn into kernel layout `layout` (see wq_packed_bytes).  The
+ * same bytes, moved; nothing is recomputed.  packed_bytes is the size of
+ * `packed` and must be >= wq_packed_bytes(...) (else WQ_ERR_INVALID_ARG).
+ * `zeros` must be NULL iff symmetric.
+ */
+wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void* zeros, int N,
+                         int K, int group_size, int symmetric, int layout, void* packed,
+                         size_t packed_bytes, wq_stream_t stream);
+
+/*
+ * wq_workspace_bytes -- workspace needed by wq_gemv_w4a16 / wq_gemm_w4a16
+ * for these sizes (split-K partial sums plus completion counters), or 0
+ * when the call needs none.  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
+ * the counters: they must be zero before the first call that uses a
+ * workspace (allocate it zero-filled), and every call that completes leaves
+ * them zero again, so one workspace serves any number of later calls of any
+ * size.  Calls that share a workspace must not run concurrently.
+ */
+#define WQ_WORKSPACE_COUNTER_BYTES 262144
+size_t wq_workspace_bytes(int M, int N, int K);
+
+/*
+ * wq_gemv_w4a16 -- the W4A16 decode linear for M = 1..8 activation rows
+ * (CUDA cores, dequantization in registers, fp32 accumulation):
+ *
+ *   y[m][n] = sum_g s16[n][g] * sum_{k in g} x'[m][k] * (q[n][k] - z[n][g])
+ *
+ * with x' = x (bf16, exact) or, when inv_act_scale is given, x'[m][k] =
+ * fp32(x[m][k]) * inv_act_scale[k] (the AWQ fold, inv_act_scale = 1/s).
+ *   x        bf16 [M][K];      inv_act_scale fp32 [K] or NULL;
+ *   packed   the weight in kernel layout `layout` (from wq_pack_layout);
+ *   y        fp32 [M][N] out;
+ *   workspace, ws_bytes: see wq_workspace_bytes (WQ_ERR_WORKSPACE_TOO_SMALL
+ *            if smaller; may be NULL when wq_workspace_bytes returns 0).
+ * The result does not depend on the GPU's scheduling: partial sums are
+ * combined in a fixed order.
+ */
+wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
+                        int N, int K, int group_size, int symmetric, int layout, float* y,
+                        void* workspace, size_t ws_bytes, wq_stream_t stream);
+
+/*
+ * wq_gemm_w4a16 -- the same linear for M = 16..64 activation rows on the
+ * tensor cores (tcgen05): weights are dequantized to bf16 tiles holding the
+ * exact integers (q - z), multiplied with x on the tensor cores with fp32
+ * accumulation per group, and each group's partial sum is scaled by s16 in
+ * fp32.  Arguments as wq_gemv_w4a16; inv_act_scale must be NULL
+ * (WQ_ERR_INVALID_ARG otherwise: the bf16 tensor-core operand cannot hold
+ * x * inv_act_scale exactly).
+ */
+wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
+                        int N, int K, int group_size, int symmetric, int layout, float* y,
+                        void* workspace, size_t ws_bytes, wq_stream_t stream);
+
+/*
+ * wq_last_device_status -- synchronize `stream`, then report and clear the
+ * device error word of the current GPU: WQ_ERR_TIMEOUT if a kernel's bounded
+ * wait gave up since the last call (its outputs are then undefined),
+ * WQ_ERR_CUDA if the stream reports a CUDA error, else WQ_OK.  The error word
+ * is shared by all streams of the GPU.
+ */
+wq_status wq_last_device_status(wq_stream_t stream);
+
+/*
+ * wq_debug_set_wait_limit_ns -- test hook, not part of the stable ABI: the
+ * time a kernel's bounded wait (on its shared-memory pipeline barriers) gives
+ * before it records WQ_ERR_TIMEOUT and returns; default 2 s, 0 is treated as
+ * 1 ns.  A tiny limit makes any wait that is not already satisfied give up at
+ * once, which exercises the timeout path without stalling the GPU.  Affects
+ * calls enqueued afterwards, from any thread.
+ */
+void wq_debug_set_wait_limit_ns(unsigned long long ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

@@ -1,0 +1,95 @@
+"""B200-native 4-bit per-group (G=128) weight quantization and W4A16 decode linear.
+
+The compute runs in ``libwq_b200.so`` (hand-written sm_100a CUDA behind the C
+ABI of ``include/wq.h``); this package only allocates device buffers with
+PyTorch and calls the ABI through :mod:`._binding`.  There is no CPU path:
+every function here raises if the library or a GPU is missing.
+
+    qw = quantize(W)                 # wq_quantize_rtn + wq_pack_layout
+    y = linear(x, qw)                # wq_gemv_w4a16 (M <= 8) / wq_gemm_w4a16 (M >= 16)
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+from . import _binding as abi
+from ._binding import WqError
+
+GROUP = abi.WQ_GROUP_SIZE
+LAYOUT = abi.WQ_LAYOUT_TILED
+
+
+def _check(status: int, where: str) -> None:
+    if status != abi.WQ_OK:
+        raise WqError(status, where)
+
+
+@dataclass
+class QuantizedWeight:
+    """A quantized weight: canonical buffers plus the kernel-layout copy."""
+    N: int
+    K: int
+    symmetric: bool
+    qweight: "object"        # torch.int32 [N][K/8] (uint32 words)
+    scales: "object"         # torch.float16 [N][K/128]
+    zeros: "object"          # torch.float16 [N][K/128] or None
+    packed: "object"         # torch.uint8 [wq_packed_bytes]
+    nonfinite_groups: int = 0
+
+
+def quantize(W, awq_scale=None, symmetric: bool = False, stream=None,
+             check_finite: bool = True) -> QuantizedWeight:
+    """Quantize a bf16 CUDA tensor W [N][K] (optionally with the AWQ scale
+    folded in) and lay it out for the linear kernels."""
+    import torch
+    N, K = W.shape
+    dev = W.device
+    qweight = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+    scales = torch.empty((N, K // GROUP), dtype=torch.float16, device=dev)
+    zeros = None if symmetric else torch.empty((N, K // GROUP), dtype=torch.float16, device=dev)
+    d_status = torch.zeros(4, dtype=torch.int32, device=dev)
+    _check(abi.wq_quantize_rtn(W, awq_scale, N, K, GROUP, symmetric, qweight, scales, zeros,
+                               d_status, stream), "wq_quantize_rtn")
+    nbytes = abi.wq_packed_bytes(N, K, GROUP, symmetric, LAYOUT)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(abi.wq_pack_layout(qweight, scales, zeros, N, K, GROUP, symmetric, LAYOUT, packed,
+                              nbytes, stream), "wq_pack_layout")
+    bad = int(d_status[0].item()) if check_finite else 0
+    return QuantizedWeight(N, K, symmetric, qweight, scales, zeros, packed, bad)
+
+
+_workspaces = {}
+
+
+def workspace_for(M: int, N: int, K: int, device):
+    """A zero-filled workspace large enough for (M, N, K), cached per device."""
+    import torch
+    need = abi.wq_workspace_bytes(M, N, K)
+    if need == 0:
+        return None, 0
+    key = (str(device),)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws, ws.numel()
+
+
+def linear(x, qw: QuantizedWeight, inv_act_scale=None, out=None, workspace=None, stream=None):
+    """y = x' dequant(W)^T as fp32 [M][N] for a bf16 CUDA tensor x [M][K]."""
+    import torch
+    M, K = x.shape
+    assert K == qw.K
+    y = out if out is not None else torch.empty((M, qw.N), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        ws, ws_bytes = workspace_for(M, qw.N, K, x.device)
+    else:
+        ws, ws_bytes = workspace, workspace.numel()
+    fn = abi.wq_gemv_w4a16 if M <= 8 else abi.wq_gemm_w4a16
+    _check(fn(x, inv_act_scale, qw.packed, M, qw.N, K, GROUP, qw.symmetric, LAYOUT, y, ws,
+              ws_bytes, stream), fn.__name__)
+    return y
+
+
+def last_device_status(stream=None) -> int:
+    return abi.wq_last_device_status(stream)

@@ -1,0 +1,257 @@
+// wq_api.cu -- the extern "C" entry points declared in include/wq.h: argument
+// validation, per-device launch state and the device error word.
+#include <atomic>
+#include <mutex>
+
+#include "wq_common.cuh"
+
+namespace wq {
+cudaError_t launch_quantize(const void* W, const float* awq, int N, int K, int sym,
+                            uint32_t* qweight, void* scales, void* zeros, int* d_status,
+                            cudaStream_t stream, int num_sms);
+cudaError_t launch_relayout(const uint32_t* qweight, const void* scales, const void* zeros,
+                            int N, int K, int sym, void* packed, cudaStream_t stream);
+size_t gemv_workspace_bytes(int M, int N, int K);
+cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, int M, int N,
+                        int K, int sym, float* y, void* workspace, int* err, int num_sms,
+                        unsigned long long wait_ns, cudaStream_t stream);
+size_t gemm_workspace_bytes(int M, int N, int K);
+cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, int sym,
+                        float* y, void* workspace, int* err, int num_sms,
+                        unsigned long long wait_ns, cudaStream_t stream);
+}  // namespace wq
+
+namespace wq {
+
+cudaError_t kernel_setup(const void* fn, size_t smem, int threads, int* ctas_per_sm) {
+  struct Entry {
+    int dev;
+    const void* fn;
+    size_t smem;
+    int per_sm;
+  };
+  static std::mutex mu;
+  static Entry cache[256];
+  static int used = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (cache[i].dev == dev && cache[i].fn == fn && cache[i].smem == smem) {
+        *ctas_per_sm = cache[i].per_sm;
+        return cudaSuccess;
+      }
+  }
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  std::lock_guard<std::mutex> lock(mu);
+  if (used < 256) cache[used++] = Entry{dev, fn, smem, per_sm};
+  *ctas_per_sm = per_sm;
+  return cudaSuccess;
+}
+
+}  // namespace wq
+
+// One error word per GPU that loads the library: kernels OR bits into it when
+// a bounded wait gives up; wq_last_device_status reads and clears it.
+__device__ int g_wq_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;   // 2 s
+
+struct DeviceState {
+  std::once_flag once;
+  int* err = nullptr;
+  int num_sms = 0;
+  cudaError_t init_error = cudaSuccess;
+};
+DeviceState g_devices[kMaxDevices];
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+
+// Per-device set-up, done once with that device current: the address of the
+// error word and the SM count.
+DeviceState* device_state(cudaError_t* e) {
+  int dev = 0;
+  *e = cudaGetDevice(&dev);
+  if (*e != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *e = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  DeviceState* d = &g_devices[dev];
+  std::call_once(d->once, [d, dev]() {
+    cudaError_t err = cudaGetSymbolAddress(reinterpret_cast<void**>(&d->err), g_wq_device_error);
+    if (err == cudaSuccess)
+      err = cudaDeviceGetAttribute(&d->num_sms, cudaDevAttrMultiProcessorCount, dev);
+    d->init_error = err;
+  });
+  *e = d->init_error;
+  return *e == cudaSuccess ? d : nullptr;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+wq_status check_dims(int N, int K, int group_size) {
+  if (N <= 0 || K <= 0) return WQ_ERR_INVALID_ARG;
+  if (group_size != WQ_GROUP_SIZE) return WQ_ERR_UNSUPPORTED_SHAPE;
+  if (K % WQ_GROUP_SIZE != 0) return WQ_ERR_UNSUPPORTED_SHAPE;
+  if (N > WQ_MAX_DIM || K > WQ_MAX_DIM) return WQ_ERR_UNSUPPORTED_SHAPE;
+  return WQ_OK;
+}
+
+wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+wq_status check_linear(const void* x, const float* inv_s, const void* packed, int M, int Mlo,
+                       int Mhi, int N, int K, int group_size, int symmetric, int layout, float* y,
+                       void* workspace, size_t ws_bytes) {
+  wq_status st = check_dims(N, K, group_size);
+  if (st != WQ_OK) return st;
+  if (M < Mlo || M > Mhi) return WQ_ERR_UNSUPPORTED_SHAPE;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (layout != WQ_LAYOUT_TILED) return WQ_ERR_INVALID_ARG;
+  if (!x || !packed || !y) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(y) || (inv_s && !aligned16(inv_s)))
+    return WQ_ERR_MISALIGNED;
+  const size_t need = wq_workspace_bytes(M, N, K);
+  if (need > 0) {
+    if (!workspace || ws_bytes < need) return WQ_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return WQ_ERR_MISALIGNED;
+  }
+  return WQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wq_status_string(int status) {
+  switch (status) {
+    case WQ_OK: return "WQ_OK";
+    case WQ_ERR_INVALID_ARG: return "WQ_ERR_INVALID_ARG";
+    case WQ_ERR_UNSUPPORTED_SHAPE: return "WQ_ERR_UNSUPPORTED_SHAPE";
+    case WQ_ERR_MISALIGNED: return "WQ_ERR_MISALIGNED";
+    case WQ_ERR_WORKSPACE_TOO_SMALL: return "WQ_ERR_WORKSPACE_TOO_SMALL";
+    case WQ_ERR_NONFINITE: return "WQ_ERR_NONFINITE";
+    case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT";
+    case WQ_ERR_CUDA: return "WQ_ERR_CUDA";
+    default: return "WQ_ERR_UNKNOWN";
+  }
+}
+
+int wq_abi_version(void) { return WQ_ABI_VERSION; }
+
+wq_status wq_quantize_rtn(const void* W, const float* awq_scale, int N, int K, int group_size,
+                          int symmetric, uint32_t* qweight, void* scales, void* zeros,
+                          int* d_status, wq_stream_t stream) {
+  wq_status st = check_dims(N, K, group_size);
+  if (st != WQ_OK) return st;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (!W || !qweight || !scales) return WQ_ERR_INVALID_ARG;
+  if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) ||
+      (zeros && !aligned16(zeros)) || (awq_scale && !aligned16(awq_scale)))
+    return WQ_ERR_MISALIGNED;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return WQ_ERR_MISALIGNED;
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_quantize(W, awq_scale, N, K, symmetric, qweight, scales, zeros,
+                                       d_status, reinterpret_cast<cudaStream_t>(stream),
+                                       d->num_sms));
+}
+
+size_t wq_packed_bytes(int N, int K, int group_size, int symmetric, int layout) {
+  if (check_dims(N, K, group_size) != WQ_OK) return 0;
+  if (layout != WQ_LAYOUT_TILED || (symmetric != 0 && symmetric != 1)) return 0;
+  return (size_t)wq::make_geom(N, K, symmetric).total;
+}
+
+wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void* zeros, int N,
+                         int K, int group_size, int symmetric, int layout, void* packed,
+                         size_t packed_bytes, wq_stream_t stream) {
+  wq_status st = check_dims(N, K, group_size);
+  if (st != WQ_OK) return st;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (layout != WQ_LAYOUT_TILED) return WQ_ERR_INVALID_ARG;
+  if (!qweight || !scales || !packed) return WQ_ERR_INVALID_ARG;
+  if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(qweight) || !aligned16(scales) || !aligned16(packed) ||
+      (zeros && !aligned16(zeros)))
+    return WQ_ERR_MISALIGNED;
+  if (packed_bytes < wq_packed_bytes(N, K, group_size, symmetric, layout))
+    return WQ_ERR_INVALID_ARG;
+  cudaError_t e;
+  if (!device_state(&e)) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_relayout(qweight, scales, zeros, N, K, symmetric, packed,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t wq_workspace_bytes(int M, int N, int K) {
+  if (N <= 0 || K <= 0 || K % WQ_GROUP_SIZE || N > WQ_MAX_DIM || K > WQ_MAX_DIM) return 0;
+  if (M >= 1 && M <= 8) return wq::gemv_workspace_bytes(M, N, K);
+  if (M >= 16 && M <= 64) return wq::gemm_workspace_bytes(M, N, K);
+  return 0;
+}
+
+wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
+                        int N, int K, int group_size, int symmetric, int layout, float* y,
+                        void* workspace, size_t ws_bytes, wq_stream_t stream) {
+  wq_status st = check_linear(x, inv_act_scale, packed, M, 1, 8, N, K, group_size, symmetric,
+                              layout, y, workspace, ws_bytes);
+  if (st != WQ_OK) return st;
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_gemv(x, inv_act_scale, packed, M, N, K, symmetric, y, workspace,
+                                   d->err, d->num_sms, g_wait_ns.load(),
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
+                        int N, int K, int group_size, int symmetric, int layout, float* y,
+                        void* workspace, size_t ws_bytes, wq_stream_t stream) {
+  wq_status st = check_linear(x, inv_act_scale, packed, M, 16, 64, N, K, group_size, symmetric,
+                              layout, y, workspace, ws_bytes);
+  if (st != WQ_OK) return st;
+  if (inv_act_scale) return WQ_ERR_INVALID_ARG;
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_gemm(x, packed, M, N, K, symmetric, y, workspace, d->err,
+                                   d->num_sms, g_wait_ns.load(),
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_last_device_status(wq_stream_t stream) {
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return WQ_ERR_CUDA;
+  e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return WQ_ERR_CUDA;
+  int word = 0;
+  e = cudaMemcpy(&word, d->err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return WQ_ERR_CUDA;
+  if (word) {
+    const int zero = 0;
+    e = cudaMemcpy(d->err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return WQ_ERR_CUDA;
+    if (word & wq::kDevErrTimeout) return WQ_ERR_TIMEOUT;
+  }
+  return WQ_OK;
+}
+
+// Test hook: the time a kernel's bounded wait gives before it records a
+// timeout (default 2 s).  Lowering it to 0 makes waits that are not already
+// satisfied give up at once, which exercises the timeout path without
+// stalling the GPU.  Not part of the stable ABI.
+void wq_debug_set_wait_limit_ns(unsigned long long ns) { g_wait_ns.store(ns ? ns : 1ull); }
+
+}  // extern "C"

@@ -155,20 +155,39 @@ def outlier_seed(cid: int, K: int) -> int:
     return 1000 * cid + 300 + (K // 1024)
 
 
+def workload_weight(cid: int, lin_index: int) -> np.ndarray:
+    lin = WORKLOADS[cid].linears[lin_index]
+    return weights(lin.N, lin.K, lin.sigma, lin.seed, lin.outlier_frac)
+
+
+def _channels(cid: int, K: int):
+    wl = WORKLOADS[cid]
+    if not wl.act_outlier_frac:
+        return None
+    return outlier_channels(K, wl.act_outlier_frac, outlier_seed(cid, K))
+
+
+def workload_activations(cid: int, lin_index: int, M: int) -> np.ndarray:
+    wl = WORKLOADS[cid]
+    K = wl.linears[lin_index].K
+    return activations(M, K, act_seed(cid, lin_index, M), _channels(cid, K), wl.act_outlier_mult)
+
+
+def workload_awq_scale(cid: int, lin_index: int):
+    """The AWQ scale of the workload's linear, or None.  The calibration rows
+    and the runtime rows share one distribution and one set of outlier
+    channels per input size K."""
+    wl = WORKLOADS[cid]
+    if not wl.awq:
+        return None
+    K = wl.linears[lin_index].K
+    X = bf16_bits_to_f32(activations(wl.calib_rows, K, calib_seed(cid, K), _channels(cid, K),
+                                     wl.calib_outlier_mult))
+    return awq_scale_from_calibration(X)
+
+
 def workload_inputs(cid: int, lin_index: int, M: int):
     """(W bits [N][K], x bits [M][K], awq_s fp32 [K] or None) for one linear of
-    a workload.  In the AWQ workload the calibration rows and the runtime rows
-    share one distribution and one set of outlier channels per input size K."""
-    wl = WORKLOADS[cid]
-    lin = wl.linears[lin_index]
-    W = weights(lin.N, lin.K, lin.sigma, lin.seed, lin.outlier_frac)
-    chans = None
-    if wl.act_outlier_frac:
-        chans = outlier_channels(lin.K, wl.act_outlier_frac, outlier_seed(cid, lin.K))
-    x = activations(M, lin.K, act_seed(cid, lin_index, M), chans, wl.act_outlier_mult)
-    s = None
-    if wl.awq:
-        X = bf16_bits_to_f32(activations(wl.calib_rows, lin.K, calib_seed(cid, lin.K), chans,
-                                         wl.calib_outlier_mult))
-        s = awq_scale_from_calibration(X)
-    return W, x, s
+    a workload."""
+    return (workload_weight(cid, lin_index), workload_activations(cid, lin_index, M),
+            workload_awq_scale(cid, lin_index))
