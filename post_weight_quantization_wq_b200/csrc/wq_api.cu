@@ -24,33 +24,45 @@ cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, 
 namespace wq {
 
 cudaError_t kernel_setup(const void* fn, size_t smem, int threads, int* ctas_per_sm) {
+  // The dynamic shared-memory limit is an attribute of the kernel, so it is
+  // only ever raised (to the largest size requested on this device so far).
   struct Entry {
     int dev;
     const void* fn;
     size_t smem;
     int per_sm;
   };
+  struct Limit {
+    int dev;
+    const void* fn;
+    size_t smem;
+  };
   static std::mutex mu;
   static Entry cache[256];
-  static int used = 0;
+  static Limit limits[128];
+  static int used = 0, nlimits = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    for (int i = 0; i < used; ++i)
-      if (cache[i].dev == dev && cache[i].fn == fn && cache[i].smem == smem) {
-        *ctas_per_sm = cache[i].per_sm;
-        return cudaSuccess;
-      }
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].dev == dev && cache[i].fn == fn && cache[i].smem == smem) {
+      *ctas_per_sm = cache[i].per_sm;
+      return cudaSuccess;
+    }
+  Limit* lim = nullptr;
+  for (int i = 0; i < nlimits; ++i)
+    if (limits[i].dev == dev && limits[i].fn == fn) lim = &limits[i];
+  if (!lim || lim->smem < smem) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (!lim && nlimits < 128) lim = &limits[nlimits++], lim->dev = dev, lim->fn = fn;
+    if (lim) lim->smem = smem;
   }
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  std::lock_guard<std::mutex> lock(mu);
   if (used < 256) cache[used++] = Entry{dev, fn, smem, per_sm};
   *ctas_per_sm = per_sm;
   return cudaSuccess;

@@ -9,26 +9,28 @@
 // section dtype、storage dtype、compute dtype).
 //
 // Design (B200, sm_100a):
-//   * persistent grid, every CTA streams a contiguous run of layout tiles
-//     (128 rows x 512 inputs: 32 KB of nibbles + 1-2 KB of fp16 metadata, one
-//     contiguous block in memory) through a ring of shared-memory stages with
-//     1-D bulk async copies (cp.async.bulk) completing on mbarriers; one
-//     producer warp issues the copies, eight consumer warps compute;
-//   * tiles are ordered slab-major, so a CTA keeps one K-slab of activations
-//     (fp32, with the AWQ factor applied once) in shared memory for many
-//     tiles;
+//   * persistent grid; CTA c owns the contiguous run [t0, t1) of the tile
+//     sequence u = b * NS + s (row tile b of 128 output rows, K-slab s of 512
+//     inputs), so it walks the slabs of one row tile after another and keeps
+//     each row's running sum in registers;
+//   * one producer warp streams every tile (32 KB of nibbles + its fp16
+//     metadata, contiguous in memory) together with the matching slab of x
+//     (and of the AWQ factor) into a ring of shared-memory stages with 1-D
+//     bulk async copies (cp.async.bulk) that complete on mbarriers; eight
+//     consumer warps compute;
 //   * dequantization in registers: a nibble at bit 4i of a word, OR-ed into
 //     the fp32 pattern of 2^(23-4i), is the float 2^(23-4i) + q (one LOP3);
-//     one packed fp32x2 subtraction of the constants gives two exact codes,
-//     and packed fp32x2 FMAs accumulate x * q; per (row, group) the sum is
-//     corrected by z * sum(x) and scaled by s16 in fp32;
-//   * a half warp owns one row: lane p covers inputs 32p..32p+31 of the slab;
-//     the 16 lanes' partial sums of several rows are combined with a
-//     transposing shuffle reduction;
-//   * split-K across slabs: every (slab, 16-row block) writes fp32 partials to
-//     the workspace; the last of the K-slabs to finish (counted with an atomic
-//     per 16-row block) adds them in slab order, so the result is the same
-//     whatever order the GPU runs the tiles in, and resets its counter.
+//     a packed fp32x2 subtraction gives two exact codes and packed fp32x2 FMAs
+//     accumulate x * q; per (row, group) the sum is corrected by z * sum(x)
+//     and scaled by the fp16 scale in fp32;
+//   * a half warp owns one row of a tile: lane p covers inputs 32p..32p+31
+//     of the slab; the 16 lanes' partial sums of several rows are combined
+//     with a transposing shuffle reduction;
+//   * a row tile whose slabs are split between CTAs (only at the ends of a
+//     CTA's run) is finished through the workspace: each piece writes its
+//     fp32 partial, and the last piece to arrive (an atomic counter per 16
+//     rows) adds the pieces in slab order and resets the counter, so y does
+//     not depend on the order the GPU runs the CTAs in;
 //   * every wait is bounded (globaltimer): on timeout the kernel records the
 //     device error word, stops issuing copies, waits (bounded) for its copies
 //     in flight and returns.
@@ -41,11 +43,11 @@ struct GemvParams {
   const uint16_t* x;       // bf16 [M][K]
   const float* inv_s;      // fp32 [K] or nullptr
   float* y;                // fp32 [M][N]
-  float* partials;         // fp32 [NS][Mp][Npad] (NS > 1)
-  unsigned* counters;      // [Npad / 16]        (NS > 1)
+  float* partials;         // fp32 [NS][MP][Npad]
+  unsigned* counters;      // one per 16 rows
   int* err;                // device error word
   Geom g;
-  int M;                   // actual rows of x / y (<= Mp)
+  int M;                   // rows of x / y (<= MP)
   long long tiles;         // NS * NB
   unsigned long long wait_ns;
   unsigned long long drain_ns;
@@ -53,9 +55,15 @@ struct GemvParams {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
-constexpr int kXPitch = kSlabK + kSlabK / 8;     // 4 pad floats per 32 inputs
+constexpr int kMaxFullTile = kTileRows * kSlabGroups * (kCodeBytesPerGroupRow + 4);
+constexpr int kInvBytes = kSlabK * 4;
 
-__device__ __forceinline__ int xpad(int k) { return k + ((k >> 5) << 2); }
+template <int MP>
+struct StageLayout {
+  static constexpr int kX = kMaxFullTile;                 // bf16 [MP][512]
+  static constexpr int kInv = kX + MP * kSlabK * 2;       // fp32 [512]
+  static constexpr int kBytes = kInv + kInvBytes;
+};
 
 // Sum v[] over the 16 lanes of a half warp.  After the call, for V >= 16 a
 // lane holds V/16 sums, v[i] being the sum of index i + (V/16)*p; for V < 16
@@ -90,21 +98,26 @@ struct ReduceMap {
   __device__ static int index(int i, int p) { return V >= 16 ? i + kPerLane * p : (p >> (4 - kLog)); }
 };
 
+// CTA that owns tile u when T tiles are split evenly over G CTAs
+// (t0(c) = floor(c*T/G)).
+__device__ __forceinline__ int owner_cta(long long u, long long T, int G) {
+  return (int)(((u + 1) * G + T - 1) / T) - 1;
+}
+
 template <int MP, int JR, int STAGES, int MINB>
 __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvParams prm) {
+  using SL = StageLayout<MP>;
   extern __shared__ __align__(128) uint8_t smem[];
   const Geom g = prm.g;
-  const long long full_tile = g.full_tile;
-  uint8_t* ring = smem;
-  float* xs = reinterpret_cast<float*>(smem + STAGES * full_tile);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(xs + MP * kXPitch);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * SL::kBytes);
   uint64_t* empty_bar = full_bar + STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty_bar + STAGES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long t0 = (long long)blockIdx.x * prm.tiles / gridDim.x;
-  const long long t1 = (long long)(blockIdx.x + 1) * prm.tiles / gridDim.x;
+  const int G = gridDim.x;
+  const long long t0 = (long long)blockIdx.x * prm.tiles / G;
+  const long long t1 = (long long)(blockIdx.x + 1) * prm.tiles / G;
   const int ntiles = (int)(t1 - t0);
 
   if (threadIdx.x == 0) {
@@ -115,6 +128,10 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
     *abort_flag = 0;
     fence_mbarrier_init();
   }
+  // Rows of x beyond M are never copied in: zero them once in every stage.
+  for (int st = 0; st < STAGES; ++st)
+    for (int i = threadIdx.x + prm.M * kSlabK / 8; i < MP * kSlabK / 8; i += blockDim.x)
+      reinterpret_cast<uint4*>(smem + st * SL::kBytes + SL::kX)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
 
   if (warp == kConsumerWarps) {
@@ -127,16 +144,23 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
           if (!mbar_wait_bounded(&empty_bar[st], ((i / STAGES) - 1) & 1, prm.wait_ns)) {
             atomicOr(prm.err, kDevErrTimeout);
             *abort_flag = 1;
-            break;
           }
         }
         if (*abort_flag) break;
-        const long long t = t0 + i;
-        const int s = (int)(t / g.NB), b = (int)(t % g.NB);
-        const uint32_t bytes = (uint32_t)tile_bytes(g, slab_groups(g, s));
-        mbar_arrive_expect_tx(&full_bar[st], bytes);
-        bulk_copy_g2s(ring + st * full_tile, prm.packed + tile_offset(g, s, b), bytes,
-                      &full_bar[st]);
+        const long long u = t0 + i;
+        const int b = (int)(u / g.NS), s = (int)(u % g.NS);
+        const int gs = slab_groups(g, s);
+        const uint32_t tbytes = (uint32_t)tile_bytes(g, gs);
+        const uint32_t xbytes = gs * kGroup * 2;
+        const uint32_t ibytes = prm.inv_s ? gs * kGroup * 4 : 0;
+        uint8_t* stage = smem + st * SL::kBytes;
+        mbar_arrive_expect_tx(&full_bar[st], tbytes + prm.M * xbytes + ibytes);
+        bulk_copy_g2s(stage, prm.packed + tile_offset(g, s, b), tbytes, &full_bar[st]);
+        for (int m = 0; m < prm.M; ++m)
+          bulk_copy_g2s(stage + SL::kX + m * kSlabK * 2, prm.x + (size_t)m * g.K + s * kSlabK,
+                        xbytes, &full_bar[st]);
+        if (ibytes)
+          bulk_copy_g2s(stage + SL::kInv, prm.inv_s + s * kSlabK, ibytes, &full_bar[st]);
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -151,52 +175,30 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
   }
 
   // ------------------------------------------------------------------ consumers
-  const int h = lane >> 4;          // row within the pair handled by this half warp
+  const int h = lane >> 4;          // row of the pair handled by this half warp
   const int p = lane & 15;          // 32-input chunk of the slab
   constexpr int V = JR * MP;
+  constexpr int kPasses = 8 / JR;
   using RM = ReduceMap<V>;
   const uint32_t E0 = 0x4B000000u, E1 = 0x49000000u, E2 = 0x47000000u, E3 = 0x45000000u;
   const float2 negE01 = make_float2(-8388608.0f, -524288.0f);
   const float2 negE23 = make_float2(-32768.0f, -2048.0f);
+  const bool awq = prm.inv_s != nullptr;
 
-  float xsum[MP];
-  int cur_s = -1;
+  float run[kPasses][RM::kPerLane];
+#pragma unroll
+  for (int a = 0; a < kPasses; ++a)
+#pragma unroll
+    for (int i2 = 0; i2 < RM::kPerLane; ++i2) run[a][i2] = 0.0f;
+  int piece_s0 = -1;                // first slab of the current row tile in this CTA
   bool aborted = false;
 
   for (int i = 0; i < ntiles; ++i) {
-    const long long t = t0 + i;
-    const int s = (int)(t / g.NB), b = (int)(t % g.NB);
+    const long long u = t0 + i;
+    const int b = (int)(u / g.NS), s = (int)(u % g.NS);
     const int gs = slab_groups(g, s);
     const int st = i % STAGES;
-
-    if (s != cur_s) {
-      // Stage this slab's activations (fp32, AWQ factor applied) once.  Every
-      // consumer warp takes part, aborted or not, so the barrier always fills.
-      named_barrier_sync(1, kConsumerWarps * 32);
-      const int kbase = s * kSlabK;
-      for (int idx = threadIdx.x; idx < MP * kSlabK; idx += kConsumerWarps * 32) {
-        const int m = idx / kSlabK, k = idx % kSlabK, kk = kbase + k;
-        float v = 0.0f;
-        if (m < prm.M && kk < g.K) {
-          v = __uint_as_float((uint32_t)prm.x[(size_t)m * g.K + kk] << 16);
-          if (prm.inv_s) v = __fmul_rn(v, __ldg(prm.inv_s + kk));
-        }
-        xs[m * kXPitch + xpad(k)] = v;
-      }
-      named_barrier_sync(1, kConsumerWarps * 32);
-#pragma unroll
-      for (int m = 0; m < MP; ++m) {
-        float a = 0.0f;
-        const float4* xp = reinterpret_cast<const float4*>(xs + m * kXPitch + xpad(32 * p));
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 v = xp[q];
-          a += (v.x + v.y) + (v.z + v.w);
-        }
-        xsum[m] = a;
-      }
-      cur_s = s;
-    }
+    if (piece_s0 < 0) piece_s0 = s;
 
     if (!aborted) {
       bool ok = mbar_wait_bounded(&full_bar[st], (i / STAGES) & 1, prm.wait_ns);
@@ -209,14 +211,17 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
     }
 
     if (!aborted) {
-      const uint8_t* tile = ring + st * full_tile;
-      const uint8_t* meta = tile + kTileRows * gs * kCodeBytesPerGroupRow;
+      const uint8_t* stage = smem + st * SL::kBytes;
+      const uint8_t* meta = stage + kTileRows * gs * kCodeBytesPerGroupRow;
+      const uint16_t* xsm = reinterpret_cast<const uint16_t*>(stage + SL::kX);
+      const float* ism = reinterpret_cast<const float*>(stage + SL::kInv);
       const int pitch = gs * kCodeBytesPerGroupRow;
       const bool active = p < gs * 4;
       const int grp = p >> 2;
 
 #pragma unroll 1
-      for (int jb = 0; jb < 8; jb += JR) {
+      for (int pass = 0; pass < kPasses; ++pass) {
+        const int jb = pass * JR;
         uint4 c[JR];
         float sc[JR], zc[JR];
 #pragma unroll
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
           sc[j] = 0.0f;
           zc[j] = 0.0f;
           if (active) {
-            c[j] = *reinterpret_cast<const uint4*>(tile + r * pitch + p * 16);
+            c[j] = *reinterpret_cast<const uint4*>(stage + r * pitch + p * 16);
             if (g.sym) {
               sc[j] = __half2float(reinterpret_cast<const __half*>(meta)[r * gs + grp]);
               zc[j] = 8.0f;
@@ -238,23 +243,38 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
           }
         }
         float2 acc[JR][MP];
+        float2 xs2[MP];
 #pragma unroll
-        for (int j = 0; j < JR; ++j)
+        for (int m = 0; m < MP; ++m) {
+          xs2[m] = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int m = 0; m < MP; ++m) acc[j][m] = make_float2(0.0f, 0.0f);
+          for (int j = 0; j < JR; ++j) acc[j][m] = make_float2(0.0f, 0.0f);
+        }
 
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
+          // x' for the 8 inputs of word wd, as fp32 pairs (bf16 -> fp32 is a shift)
           float2 xv[MP][4];
+          float4 ia = make_float4(1.f, 1.f, 1.f, 1.f), ib = ia;
+          if (awq && active) {
+            ia = *reinterpret_cast<const float4*>(ism + 32 * p + 8 * wd);
+            ib = *reinterpret_cast<const float4*>(ism + 32 * p + 8 * wd + 4);
+          }
 #pragma unroll
           for (int m = 0; m < MP; ++m) {
-            const float4* xp =
-                reinterpret_cast<const float4*>(xs + m * kXPitch + xpad(32 * p + 8 * wd));
-            const float4 a = xp[0], bq = xp[1];
-            xv[m][0] = make_float2(a.x, a.y);
-            xv[m][1] = make_float2(a.z, a.w);
-            xv[m][2] = make_float2(bq.x, bq.y);
-            xv[m][3] = make_float2(bq.z, bq.w);
+            const uint4 xb = *reinterpret_cast<const uint4*>(xsm + m * kSlabK + 32 * p + 8 * wd);
+            xv[m][0] = make_float2(__uint_as_float(xb.x << 16), __uint_as_float(xb.x & 0xFFFF0000u));
+            xv[m][1] = make_float2(__uint_as_float(xb.y << 16), __uint_as_float(xb.y & 0xFFFF0000u));
+            xv[m][2] = make_float2(__uint_as_float(xb.z << 16), __uint_as_float(xb.z & 0xFFFF0000u));
+            xv[m][3] = make_float2(__uint_as_float(xb.w << 16), __uint_as_float(xb.w & 0xFFFF0000u));
+            if (awq) {
+              xv[m][0] = __fmul2_rn(xv[m][0], make_float2(ia.x, ia.y));
+              xv[m][1] = __fmul2_rn(xv[m][1], make_float2(ia.z, ia.w));
+              xv[m][2] = __fmul2_rn(xv[m][2], make_float2(ib.x, ib.y));
+              xv[m][3] = __fmul2_rn(xv[m][3], make_float2(ib.z, ib.w));
+            }
+            xs2[m] = __fadd2_rn(xs2[m], __fadd2_rn(__fadd2_rn(xv[m][0], xv[m][1]),
+                                                 __fadd2_rn(xv[m][2], xv[m][3])));
           }
 #pragma unroll
           for (int j = 0; j < JR; ++j) {
@@ -284,60 +304,86 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
           }
         }
 
-        // y partial of (row, m) over this lane's 32 inputs:
-        //   s16 * (sum x*q - z * sum x)
+        // partial of (row, m) over this lane's 32 inputs: s16 * (sum x*q - z * sum x)
         float v[V];
 #pragma unroll
         for (int j = 0; j < JR; ++j)
 #pragma unroll
           for (int m = 0; m < MP; ++m)
-            v[j * MP + m] = active ? sc[j] * ((acc[j][m].x + acc[j][m].y) - zc[j] * xsum[m]) : 0.0f;
+            v[j * MP + m] = active ? sc[j] * ((acc[j][m].x + acc[j][m].y) -
+                                              zc[j] * (xs2[m].x + xs2[m].y))
+                                   : 0.0f;
         half_transpose_reduce<V>(v, p);
-
-        if (RM::writer(p)) {
 #pragma unroll
-          for (int i2 = 0; i2 < RM::kPerLane; ++i2) {
-            const int idx = RM::index(i2, p);
-            const int j = idx / MP, m = idx % MP;
-            const int n = b * kTileRows + warp * 16 + 2 * (jb + j) + h;
-            if (m < prm.M) {
-              if (g.NS == 1) {
-                if (n < g.N) prm.y[(size_t)m * g.N + n] = v[i2];
-              } else {
-                prm.partials[((size_t)s * MP + m) * g.Npad + n] = v[i2];
-              }
-            }
-          }
-        }
+        for (int i2 = 0; i2 < RM::kPerLane; ++i2) run[pass][i2] += v[i2];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
 
-    // ---- split-K completion: the last slab to finish a 16-row block sums it
-    if (g.NS > 1) {
-      __threadfence();
-      __syncwarp();
-      unsigned prev = 0;
-      unsigned* ctr = prm.counters + (size_t)b * (kTileRows / kRowsPerCounter) + warp;
-      if (lane == 0) prev = atomicAdd(ctr, 1u);
-      prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-      if (prev == (unsigned)(g.NS - 1)) {
-        __threadfence();
-        if (!aborted) {
-          for (int e = lane; e < kRowsPerCounter * prm.M; e += 32) {
-            const int n = b * kTileRows + warp * kRowsPerCounter + (e % kRowsPerCounter);
-            const int m = e / kRowsPerCounter;
-            float acc = 0.0f;
-            const float* src = prm.partials + (size_t)m * g.Npad + n;
-            const size_t slab_stride = (size_t)MP * g.Npad;
-#pragma unroll 8
-            for (int s2 = 0; s2 < g.NS; ++s2) acc += __ldcg(src + s2 * slab_stride);
-            if (n < g.N) prm.y[(size_t)m * g.N + n] = acc;
-          }
+    // ---- end of this CTA's piece of row tile b: write y or a partial
+    const bool piece_end = (s == g.NS - 1) || (i == ntiles - 1);
+    if (piece_end) {
+      const bool whole = (piece_s0 == 0) && (s == g.NS - 1);
+      if (whole) {
+        if (!aborted && RM::writer(p)) {
+#pragma unroll
+          for (int pass = 0; pass < kPasses; ++pass)
+#pragma unroll
+            for (int i2 = 0; i2 < RM::kPerLane; ++i2) {
+              const int idx = RM::index(i2, p);
+              const int j = idx / MP, m = idx % MP;
+              const int n = b * kTileRows + warp * 16 + 2 * (pass * JR + j) + h;
+              if (m < prm.M && n < g.N) prm.y[(size_t)m * g.N + n] = run[pass][i2];
+            }
         }
-        if (lane == 0) *ctr = 0u;
+      } else {
+        // Partial piece: its slot is its first slab.
+        if (!aborted && RM::writer(p)) {
+#pragma unroll
+          for (int pass = 0; pass < kPasses; ++pass)
+#pragma unroll
+            for (int i2 = 0; i2 < RM::kPerLane; ++i2) {
+              const int idx = RM::index(i2, p);
+              const int j = idx / MP, m = idx % MP;
+              const int n = b * kTileRows + warp * 16 + 2 * (pass * JR + j) + h;
+              if (m < prm.M)
+                prm.partials[((size_t)piece_s0 * MP + m) * g.Npad + n] = run[pass][i2];
+            }
+        }
+        __threadfence();
+        __syncwarp();
+        const long long ub = (long long)b * g.NS;
+        const int c_first = owner_cta(ub, prm.tiles, G);
+        const int c_last = owner_cta(ub + g.NS - 1, prm.tiles, G);
+        unsigned prev = 0;
+        unsigned* ctr = prm.counters + (size_t)b * (kTileRows / kRowsPerCounter) + warp;
+        if (lane == 0) prev = atomicAdd(ctr, 1u);
+        prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+        if (prev == (unsigned)(c_last - c_first)) {
+          // Last piece: add all pieces in slab order, reset the counter.
+          __threadfence();
+          if (!aborted) {
+            for (int e = lane; e < kRowsPerCounter * prm.M; e += 32) {
+              const int n = b * kTileRows + warp * kRowsPerCounter + (e % kRowsPerCounter);
+              const int m = e / kRowsPerCounter;
+              float tot = 0.0f;
+              for (int c2 = c_first; c2 <= c_last; ++c2) {
+                const long long tc = (long long)c2 * prm.tiles / G;
+                const int sa = (int)((tc > ub ? tc : ub) - ub);
+                tot += __ldcg(prm.partials + ((size_t)sa * MP + m) * g.Npad + n);
+              }
+              if (n < g.N) prm.y[(size_t)m * g.N + n] = tot;
+            }
+          }
+          if (lane == 0) *ctr = 0u;
+        }
       }
+#pragma unroll
+      for (int a = 0; a < kPasses; ++a)
+#pragma unroll
+        for (int i2 = 0; i2 < RM::kPerLane; ++i2) run[a][i2] = 0.0f;
+      piece_s0 = -1;
     }
   }
 }
@@ -346,32 +392,32 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
 
 struct GemvConfig {
   const void* fn;
-  int stages;
   size_t smem;
 };
 
 template <int MP, int JR, int STAGES, int MINB>
-static GemvConfig gemv_config(const Geom& g) {
+static GemvConfig gemv_config() {
   GemvConfig c;
   c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JR, STAGES, MINB>);
-  c.stages = STAGES;
-  c.smem = (size_t)STAGES * g.full_tile + (size_t)MP * kXPitch * sizeof(float) +
-           2 * STAGES * sizeof(uint64_t) + 16;
+  c.smem = (size_t)STAGES * StageLayout<MP>::kBytes + 2 * STAGES * sizeof(uint64_t) + 16;
   return c;
 }
 
-static GemvConfig pick_gemv(int M, const Geom& g) {
-  if (M <= 1) return gemv_config<1, 8, 3, 2>(g);
-  if (M <= 2) return gemv_config<2, 4, 3, 2>(g);
-  if (M <= 4) return gemv_config<4, 4, 4, 1>(g);
-  return gemv_config<8, 2, 4, 1>(g);
+static int padded_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+
+static GemvConfig pick_gemv(int M) {
+  switch (padded_m(M)) {
+    case 1: return gemv_config<1, 8, 3, 2>();
+    case 2: return gemv_config<2, 4, 3, 2>();
+    case 4: return gemv_config<4, 4, 4, 1>();
+    default: return gemv_config<8, 2, 4, 1>();
+  }
 }
 
 size_t gemv_workspace_bytes(int M, int N, int K) {
   const Geom g = make_geom(N, K, 1);
   if (g.NS <= 1) return 0;
-  const int MP = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
-  return (size_t)kCounterBytes + (size_t)g.NS * MP * g.Npad * sizeof(float);
+  return (size_t)kCounterBytes + (size_t)g.NS * padded_m(M) * g.Npad * sizeof(float);
 }
 
 cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, int M, int N,
@@ -392,7 +438,7 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   prm.wait_ns = wait_ns;
   prm.drain_ns = 1000000000ull;
 
-  const GemvConfig c = pick_gemv(M, prm.g);
+  const GemvConfig c = pick_gemv(M);
   int per_sm = 0;
   cudaError_t e = kernel_setup(c.fn, c.smem, kGemvThreads, &per_sm);
   if (e != cudaSuccess) return e;
