@@ -13,19 +13,24 @@
 //     sequence u = b * NS + s (row tile b of 128 output rows, K-slab s of 512
 //     inputs), so it walks the slabs of one row tile after another and keeps
 //     each row's running sum in registers;
-//   * one producer warp streams every tile (32 KB of nibbles + its fp16
-//     metadata, contiguous in memory) together with the matching slab of x
-//     (and of the AWQ factor) into a ring of shared-memory stages with 1-D
-//     bulk async copies (cp.async.bulk) that complete on mbarriers; eight
-//     consumer warps compute;
-//   * dequantization in registers: a nibble at bit 4i of a word, OR-ed into
-//     the fp32 pattern of 2^(23-4i), is the float 2^(23-4i) + q (one LOP3);
-//     a packed fp32x2 subtraction gives two exact codes and packed fp32x2 FMAs
-//     accumulate x * q; per (row, group) the sum is corrected by z * sum(x)
-//     and scaled by the fp16 scale in fp32;
-//   * a half warp owns one row of a tile: lane p covers inputs 32p..32p+31
-//     of the slab; the 16 lanes' partial sums of several rows are combined
-//     with a transposing shuffle reduction;
+//   * a producer warp streams every tile (32 KB of nibbles + its fp16
+//     metadata, contiguous in memory) into a ring of shared-memory stages with
+//     one 1-D bulk async copy (cp.async.bulk) completing on an mbarrier, and
+//     prepares the tile's activation slab once for the whole CTA: bf16 x plus
+//     fp32 sums of x per 64 inputs (mixed path), or fp32 x * (1/s) (packed
+//     path); eight consumer warps compute;
+//   * dequantization in registers: the nibbles at bits 4i and 16+4i of a word,
+//     masked and OR-ed into 0x43004300, are two bf16 values 128 + q (one LOP3
+//     for two codes, exact).  Mixed path (no activation scale, M <= 4): the
+//     bf16 codes meet the bf16 activations in sm_100's mixed-precision FMA
+//     (bf16 x bf16 + fp32, exact product), and each (row, group) sum is
+//     corrected by (128 + z) * sum(x) and scaled by the fp16 scale in fp32.
+//     Packed path (AWQ fold, M = 8): each 128 + q is widened to the fp32 code
+//     q - z by a mixed-precision add, and packed fp32x2 FMAs multiply it with
+//     the fp32 activations;
+//   * 8 lanes share a row of a tile, lane p covering inputs 64p..64p+63 of
+//     the slab; their partial sums of several rows are combined with a
+//     transposing shuffle reduction;
 //   * a row tile whose slabs are split between CTAs (only at the ends of a
 //     CTA's run) is finished through the workspace: each piece writes its
 //     fp32 partial, and the last piece to arrive (an atomic counter per 16
@@ -56,23 +61,27 @@ struct GemvParams {
 constexpr int kConsumerWarps = 8;
 constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxFullTile = kTileRows * kSlabGroups * (kCodeBytesPerGroupRow + 4);
-constexpr int kInvBytes = kSlabK * 4;
+constexpr int kLaneK = 64;                          // inputs of one row per lane
+constexpr int kChunks = kSlabK / kLaneK;            // 8 lanes per row
+constexpr int kXbChunk = kLaneK * 2 + 16;           // bf16 chunk + pad (conflict-free)
+constexpr int kXfChunk = kLaneK * 4 + 16;           // fp32 chunk + pad
 
-template <int MP>
+template <int MP, bool MIXED>
 struct StageLayout {
-  static constexpr int kX = kMaxFullTile;                 // bf16 [MP][512]
-  static constexpr int kInv = kX + MP * kSlabK * 2;       // fp32 [512]
-  static constexpr int kBytes = kInv + kInvBytes;
+  static constexpr int kX = kMaxFullTile;
+  static constexpr int kXRow = kChunks * (MIXED ? kXbChunk : kXfChunk);
+  static constexpr int kXsum = kX + MP * kXRow;                       // fp32 [MP][8]
+  static constexpr int kBytes = kXsum + (MIXED ? MP * kChunks * 4 : 0);
 };
 
-// Sum v[] over the 16 lanes of a half warp.  After the call, for V >= 16 a
-// lane holds V/16 sums, v[i] being the sum of index i + (V/16)*p; for V < 16
-// a lane holds one sum, of index p >> (4 - log2 V).  (p = lane & 15.)
-template <int V>
-__device__ __forceinline__ void half_transpose_reduce(float (&v)[V], int p) {
+// Sum v[] over the L lanes (L = 8 or 16, lane index p) of a lane group.
+// Afterwards, for V >= L a lane holds V/L sums, v[i] being the sum of index
+// i + (V/L)*p; for V < L a lane holds one sum, of index p >> (log2 L - log2 V).
+template <int V, int L>
+__device__ __forceinline__ void group_transpose_reduce(float (&v)[V], int p) {
   int C = V;
 #pragma unroll
-  for (int mk = 8; mk >= 1; mk >>= 1) {
+  for (int mk = L / 2; mk >= 1; mk >>= 1) {
     if (C >= 2) {
       const bool upper = (p & mk) != 0;
 #pragma unroll
@@ -90,13 +99,61 @@ __device__ __forceinline__ void half_transpose_reduce(float (&v)[V], int p) {
   }
 }
 
-template <int V>
-struct ReduceMap {
-  static constexpr int kLog = (V >= 16) ? 4 : (V >= 8 ? 3 : (V >= 4 ? 2 : (V >= 2 ? 1 : 0)));
-  static constexpr int kPerLane = (V >= 16) ? V / 16 : 1;
-  __device__ static bool writer(int p) { return V >= 16 || (p & ((16 >> kLog) - 1)) == 0; }
-  __device__ static int index(int i, int p) { return V >= 16 ? i + kPerLane * p : (p >> (4 - kLog)); }
+__host__ __device__ constexpr int ilog2c(int v) { return v <= 1 ? 0 : 1 + ilog2c(v / 2); }
+
+template <int V, int L>
+struct GroupMap {
+  static constexpr int kPerLane = (V >= L) ? V / L : 1;
+  static constexpr int kShift = (V >= L) ? 0 : ilog2c(L) - ilog2c(V);
+  __device__ static bool writer(int p) { return V >= L || (p & ((1 << kShift) - 1)) == 0; }
+  __device__ static int index(int i, int p) { return V >= L ? i + kPerLane * p : (p >> kShift); }
 };
+
+// Two bf16 values 128 + q of the nibbles at bits [4i, 4i+4) and [16+4i, 20+4i)
+// of w (exact: 128..143 are bf16 integers).
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) {
+  return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+}
+
+// acc += x_k * (128 + q_k) for the 8 inputs of one word, with sm_100's
+// mixed-precision FMA (bf16 * bf16 + fp32, one rounding, exact product).
+// xw holds the 8 bf16 activations as pairs (x0,x1) (x2,x3) (x4,x5) (x6,x7).
+__device__ __forceinline__ void mixed_word(uint32_t w, const uint4& xw, float& a0, float& a1) {
+  const uint32_t v0 = nib_pair(w, 0), v1 = nib_pair(w, 1), v2 = nib_pair(w, 2),
+                 v3 = nib_pair(w, 3);   // vi = (q_i, q_{i+4})
+  asm("{\n\t.reg .b16 q0, q4, q1, q5, q2, q6, q3, q7, x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
+      "mov.b32 {q0, q4}, %2;\n\tmov.b32 {q1, q5}, %3;\n\t"
+      "mov.b32 {q2, q6}, %4;\n\tmov.b32 {q3, q7}, %5;\n\t"
+      "mov.b32 {x0, x1}, %6;\n\tmov.b32 {x2, x3}, %7;\n\t"
+      "mov.b32 {x4, x5}, %8;\n\tmov.b32 {x6, x7}, %9;\n\t"
+      "fma.rn.f32.bf16 %0, q0, x0, %0;\n\tfma.rn.f32.bf16 %1, q1, x1, %1;\n\t"
+      "fma.rn.f32.bf16 %0, q2, x2, %0;\n\tfma.rn.f32.bf16 %1, q3, x3, %1;\n\t"
+      "fma.rn.f32.bf16 %0, q4, x4, %0;\n\tfma.rn.f32.bf16 %1, q5, x5, %1;\n\t"
+      "fma.rn.f32.bf16 %0, q6, x6, %0;\n\tfma.rn.f32.bf16 %1, q7, x7, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(v0), "r"(v1), "r"(v2), "r"(v3), "r"(xw.x), "r"(xw.y), "r"(xw.z), "r"(xw.w));
+}
+
+// The 8 codes of one word as exact fp32 (q - z) pairs, in input order:
+// f32(128 + q) + cz with cz = -(128 + z), by the mixed-precision add.
+__device__ __forceinline__ void widen_word(uint32_t w, float cz, float2& d01, float2& d23,
+                                           float2& d45, float2& d67) {
+  const uint32_t v0 = nib_pair(w, 0), v1 = nib_pair(w, 1), v2 = nib_pair(w, 2),
+                 v3 = nib_pair(w, 3);
+  asm("{\n\t.reg .b16 q0, q4, q1, q5, q2, q6, q3, q7;\n\t"
+      "mov.b32 {q0, q4}, %8;\n\tmov.b32 {q1, q5}, %9;\n\t"
+      "mov.b32 {q2, q6}, %10;\n\tmov.b32 {q3, q7}, %11;\n\t"
+      "add.rn.f32.bf16 %0, q0, %12;\n\tadd.rn.f32.bf16 %1, q1, %12;\n\t"
+      "add.rn.f32.bf16 %2, q2, %12;\n\tadd.rn.f32.bf16 %3, q3, %12;\n\t"
+      "add.rn.f32.bf16 %4, q4, %12;\n\tadd.rn.f32.bf16 %5, q5, %12;\n\t"
+      "add.rn.f32.bf16 %6, q6, %12;\n\tadd.rn.f32.bf16 %7, q7, %12;\n\t}"
+      : "=f"(d01.x), "=f"(d01.y), "=f"(d23.x), "=f"(d23.y), "=f"(d45.x), "=f"(d45.y),
+        "=f"(d67.x), "=f"(d67.y)
+      : "r"(v0), "r"(v1), "r"(v2), "r"(v3), "f"(cz));
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
 // CTA that owns tile u when T tiles are split evenly over G CTAs
 // (t0(c) = floor(c*T/G)).
@@ -104,9 +161,74 @@ __device__ __forceinline__ int owner_cta(long long u, long long T, int G) {
   return (int)(((u + 1) * G + T - 1) / T) - 1;
 }
 
-template <int MP, int JR, int STAGES, int MINB>
+// The producer lanes' share of one activation slab: lane l holds inputs
+// 16l .. 16l+15 of the slab for every row of x (and of the AWQ factor).
+template <int MP, bool MIXED>
+struct XSlice {
+  uint4 xb[MP][2];
+  float4 inv[MIXED ? 1 : 4];
+};
+
+template <int MP, bool MIXED>
+__device__ __forceinline__ void load_x_slice(XSlice<MP, MIXED>& xs, const GemvParams& prm, int s,
+                                             int lane) {
+  const int k = s * kSlabK + 16 * lane;
+  const bool ok = k < prm.g.K;
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+    xs.xb[m][0] = make_uint4(0, 0, 0, 0);
+    xs.xb[m][1] = make_uint4(0, 0, 0, 0);
+    if (ok && m < prm.M) {
+      const uint4* src = reinterpret_cast<const uint4*>(prm.x + (size_t)m * prm.g.K + k);
+      xs.xb[m][0] = __ldg(src);
+      xs.xb[m][1] = __ldg(src + 1);
+    }
+  }
+  if constexpr (!MIXED) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      xs.inv[q] = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (ok && prm.inv_s) xs.inv[q] = __ldg(reinterpret_cast<const float4*>(prm.inv_s + k) + q);
+    }
+  }
+}
+
+template <int MP, bool MIXED>
+__device__ __forceinline__ void store_x_slice(const XSlice<MP, MIXED>& xs, uint8_t* stage,
+                                              const GemvParams& prm, int lane) {
+  using SL = StageLayout<MP, MIXED>;
+  const int c = lane >> 2, sub = lane & 3;      // 64-input chunk and quarter of it
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+    if (m >= prm.M) break;
+    const uint32_t r[8] = {xs.xb[m][0].x, xs.xb[m][0].y, xs.xb[m][0].z, xs.xb[m][0].w,
+                           xs.xb[m][1].x, xs.xb[m][1].y, xs.xb[m][1].z, xs.xb[m][1].w};
+    if constexpr (MIXED) {
+      uint4* dst = reinterpret_cast<uint4*>(stage + SL::kX + m * SL::kXRow + c * kXbChunk + sub * 32);
+      dst[0] = xs.xb[m][0];
+      dst[1] = xs.xb[m][1];
+      float sum = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sum += bf16_lo(r[q]) + bf16_hi(r[q]);
+      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+      if (sub == 0) reinterpret_cast<float*>(stage + SL::kXsum)[m * kChunks + c] = sum;
+    } else {
+      float4* dst = reinterpret_cast<float4*>(stage + SL::kX + m * SL::kXRow + c * kXfChunk + sub * 64);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 iv = xs.inv[q];
+        dst[q] = make_float4(__fmul_rn(bf16_lo(r[2 * q]), iv.x), __fmul_rn(bf16_hi(r[2 * q]), iv.y),
+                             __fmul_rn(bf16_lo(r[2 * q + 1]), iv.z),
+                             __fmul_rn(bf16_hi(r[2 * q + 1]), iv.w));
+      }
+    }
+  }
+}
+
+template <int MP, int JQ, int STAGES, int MINB, bool MIXED>
 __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvParams prm) {
-  using SL = StageLayout<MP>;
+  using SL = StageLayout<MP, MIXED>;
   extern __shared__ __align__(128) uint8_t smem[];
   const Geom g = prm.g;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * SL::kBytes);
@@ -122,74 +244,70 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full_bar[i], 1);
+      mbar_init(&full_bar[i], 1 + 32);           // producer's expect_tx + its 32 lanes
       mbar_init(&empty_bar[i], kConsumerWarps);
     }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  // Rows of x beyond M are never copied in: zero them once in every stage.
+  // Rows of x beyond M are never written: zero every stage's activation area once.
   for (int st = 0; st < STAGES; ++st)
-    for (int i = threadIdx.x + prm.M * kSlabK / 8; i < MP * kSlabK / 8; i += blockDim.x)
+    for (int i = threadIdx.x; i < (SL::kBytes - SL::kX) / 16; i += blockDim.x)
       reinterpret_cast<uint4*>(smem + st * SL::kBytes + SL::kX)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
 
   if (warp == kConsumerWarps) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i % STAGES;
-        if (i >= STAGES) {
-          if (!mbar_wait_bounded(&empty_bar[st], ((i / STAGES) - 1) & 1, prm.wait_ns)) {
-            atomicOr(prm.err, kDevErrTimeout);
-            *abort_flag = 1;
-          }
+    int issued = 0;
+    XSlice<MP, MIXED> xs;
+    if (ntiles > 0) load_x_slice<MP, MIXED>(xs, prm, (int)(t0 % g.NS), lane);
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % STAGES;
+      bool ok = true;
+      if (i >= STAGES) ok = mbar_wait_bounded(&empty_bar[st], ((i / STAGES) - 1) & 1, prm.wait_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
+      if (!ok) {
+        if (lane == 0) {
+          atomicOr(prm.err, kDevErrTimeout);
+          *abort_flag = 1;
         }
-        if (*abort_flag) break;
-        const long long u = t0 + i;
-        const int b = (int)(u / g.NS), s = (int)(u % g.NS);
-        const int gs = slab_groups(g, s);
-        const uint32_t tbytes = (uint32_t)tile_bytes(g, gs);
-        const uint32_t xbytes = gs * kGroup * 2;
-        const uint32_t ibytes = prm.inv_s ? gs * kGroup * 4 : 0;
-        uint8_t* stage = smem + st * SL::kBytes;
-        mbar_arrive_expect_tx(&full_bar[st], tbytes + prm.M * xbytes + ibytes);
-        bulk_copy_g2s(stage, prm.packed + tile_offset(g, s, b), tbytes, &full_bar[st]);
-        for (int m = 0; m < prm.M; ++m)
-          bulk_copy_g2s(stage + SL::kX + m * kSlabK * 2, prm.x + (size_t)m * g.K + s * kSlabK,
-                        xbytes, &full_bar[st]);
-        if (ibytes)
-          bulk_copy_g2s(stage + SL::kInv, prm.inv_s + s * kSlabK, ibytes, &full_bar[st]);
-        issued = i + 1;
+        break;
       }
-      if (*abort_flag) {
-        // Wait (bounded) for every copy still in flight before the CTA exits.
-        for (int st = 0; st < STAGES && st < issued; ++st) {
-          const int uses = (issued - 1 - st) / STAGES + 1;   // copies issued on stage st
-          mbar_wait_bounded(&full_bar[st], (uses - 1) & 1, prm.drain_ns);
-        }
+      const long long u = t0 + i;
+      const int b = (int)(u / g.NS), s = (int)(u % g.NS);
+      uint8_t* stage = smem + st * SL::kBytes;
+      if (lane == 0) {
+        const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, s));
+        mbar_arrive_expect_tx(&full_bar[st], tbytes);
+        bulk_copy_g2s(stage, prm.packed + tile_offset(g, s, b), tbytes, &full_bar[st]);
+      }
+      store_x_slice<MP, MIXED>(xs, stage, prm, lane);
+      mbar_arrive(&full_bar[st]);
+      issued = i + 1;
+      if (i + 1 < ntiles) load_x_slice<MP, MIXED>(xs, prm, (int)((u + 1) % g.NS), lane);
+    }
+    if (lane == 0 && *abort_flag) {
+      // Wait (bounded) for every copy still in flight before the CTA exits.
+      for (int st = 0; st < STAGES && st < issued; ++st) {
+        const int uses = (issued - 1 - st) / STAGES + 1;   // copies issued on stage st
+        mbar_wait_bounded(&full_bar[st], (uses - 1) & 1, prm.drain_ns);
       }
     }
     return;
   }
 
   // ------------------------------------------------------------------ consumers
-  const int h = lane >> 4;          // row of the pair handled by this half warp
-  const int p = lane & 15;          // 32-input chunk of the slab
-  constexpr int V = JR * MP;
-  constexpr int kPasses = 8 / JR;
-  using RM = ReduceMap<V>;
-  const uint32_t E0 = 0x4B000000u, E1 = 0x49000000u, E2 = 0x47000000u, E3 = 0x45000000u;
-  const float2 negE01 = make_float2(-8388608.0f, -524288.0f);
-  const float2 negE23 = make_float2(-32768.0f, -2048.0f);
-  const bool awq = prm.inv_s != nullptr;
+  const int rq = lane >> 3;         // row of the quad handled by this lane group
+  const int p = lane & 7;           // 64-input chunk of the slab
+  constexpr int V = JQ * MP;
+  constexpr int kPasses = 4 / JQ;
+  using GM = GroupMap<V, 8>;
 
-  float run[kPasses][RM::kPerLane];
+  float run[kPasses][GM::kPerLane];
 #pragma unroll
   for (int a = 0; a < kPasses; ++a)
 #pragma unroll
-    for (int i2 = 0; i2 < RM::kPerLane; ++i2) run[a][i2] = 0.0f;
+    for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[a][i2] = 0.0f;
   int piece_s0 = -1;                // first slab of the current row tile in this CTA
   bool aborted = false;
 
@@ -213,25 +331,25 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
     if (!aborted) {
       const uint8_t* stage = smem + st * SL::kBytes;
       const uint8_t* meta = stage + kTileRows * gs * kCodeBytesPerGroupRow;
-      const uint16_t* xsm = reinterpret_cast<const uint16_t*>(stage + SL::kX);
-      const float* ism = reinterpret_cast<const float*>(stage + SL::kInv);
       const int pitch = gs * kCodeBytesPerGroupRow;
-      const bool active = p < gs * 4;
-      const int grp = p >> 2;
+      const bool active = p < 2 * gs;
+      const int grp = p >> 1;
+      float xsum[MP];
+      if constexpr (MIXED) {
+#pragma unroll
+        for (int m = 0; m < MP; ++m)
+          xsum[m] = reinterpret_cast<const float*>(stage + SL::kXsum)[m * kChunks + p];
+      }
 
 #pragma unroll 1
       for (int pass = 0; pass < kPasses; ++pass) {
-        const int jb = pass * JR;
-        uint4 c[JR];
-        float sc[JR], zc[JR];
+        float sc[JQ], zc[JQ];
 #pragma unroll
-        for (int j = 0; j < JR; ++j) {
-          const int r = warp * 16 + 2 * (jb + j) + h;
-          c[j] = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < JQ; ++j) {
+          const int r = warp * 16 + 4 * (pass * JQ + j) + rq;
           sc[j] = 0.0f;
           zc[j] = 0.0f;
           if (active) {
-            c[j] = *reinterpret_cast<const uint4*>(stage + r * pitch + p * 16);
             if (g.sym) {
               sc[j] = __half2float(reinterpret_cast<const __half*>(meta)[r * gs + grp]);
               zc[j] = 8.0f;
@@ -242,80 +360,107 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
             }
           }
         }
-        float2 acc[JR][MP];
-        float2 xs2[MP];
-#pragma unroll
-        for (int m = 0; m < MP; ++m) {
-          xs2[m] = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int j = 0; j < JR; ++j) acc[j][m] = make_float2(0.0f, 0.0f);
-        }
-
-#pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          // x' for the 8 inputs of word wd, as fp32 pairs (bf16 -> fp32 is a shift)
-          float2 xv[MP][4];
-          float4 ia = make_float4(1.f, 1.f, 1.f, 1.f), ib = ia;
-          if (awq && active) {
-            ia = *reinterpret_cast<const float4*>(ism + 32 * p + 8 * wd);
-            ib = *reinterpret_cast<const float4*>(ism + 32 * p + 8 * wd + 4);
-          }
-#pragma unroll
-          for (int m = 0; m < MP; ++m) {
-            const uint4 xb = *reinterpret_cast<const uint4*>(xsm + m * kSlabK + 32 * p + 8 * wd);
-            xv[m][0] = make_float2(__uint_as_float(xb.x << 16), __uint_as_float(xb.x & 0xFFFF0000u));
-            xv[m][1] = make_float2(__uint_as_float(xb.y << 16), __uint_as_float(xb.y & 0xFFFF0000u));
-            xv[m][2] = make_float2(__uint_as_float(xb.z << 16), __uint_as_float(xb.z & 0xFFFF0000u));
-            xv[m][3] = make_float2(__uint_as_float(xb.w << 16), __uint_as_float(xb.w & 0xFFFF0000u));
-            if (awq) {
-              xv[m][0] = __fmul2_rn(xv[m][0], make_float2(ia.x, ia.y));
-              xv[m][1] = __fmul2_rn(xv[m][1], make_float2(ia.z, ia.w));
-              xv[m][2] = __fmul2_rn(xv[m][2], make_float2(ib.x, ib.y));
-              xv[m][3] = __fmul2_rn(xv[m][3], make_float2(ib.z, ib.w));
-            }
-            xs2[m] = __fadd2_rn(xs2[m], __fadd2_rn(__fadd2_rn(xv[m][0], xv[m][1]),
-                                                 __fadd2_rn(xv[m][2], xv[m][3])));
-          }
-#pragma unroll
-          for (int j = 0; j < JR; ++j) {
-            const uint32_t lo = wd == 0 ? c[j].x : wd == 1 ? c[j].y : wd == 2 ? c[j].z : c[j].w;
-            const uint32_t hi = lo >> 16;
-            const float2 q01 = __fadd2_rn(make_float2(__uint_as_float((lo & 0xFu) | E0),
-                                                      __uint_as_float((lo & 0xF0u) | E1)),
-                                          negE01);
-            const float2 q23 = __fadd2_rn(make_float2(__uint_as_float((lo & 0xF00u) | E2),
-                                                      __uint_as_float((lo & 0xF000u) | E3)),
-                                          negE23);
-            const float2 q45 = __fadd2_rn(make_float2(__uint_as_float((hi & 0xFu) | E0),
-                                                      __uint_as_float((hi & 0xF0u) | E1)),
-                                          negE01);
-            const float2 q67 = __fadd2_rn(make_float2(__uint_as_float((hi & 0xF00u) | E2),
-                                                      __uint_as_float((hi & 0xF000u) | E3)),
-                                          negE23);
-#pragma unroll
-            for (int m = 0; m < MP; ++m) {
-              float2 a = acc[j][m];
-              a = __ffma2_rn(q01, xv[m][0], a);
-              a = __ffma2_rn(q23, xv[m][1], a);
-              a = __ffma2_rn(q45, xv[m][2], a);
-              a = __ffma2_rn(q67, xv[m][3], a);
-              acc[j][m] = a;
-            }
-          }
-        }
-
-        // partial of (row, m) over this lane's 32 inputs: s16 * (sum x*q - z * sum x)
         float v[V];
+        // The lane's 64 inputs of a row are two 16-byte halves of 4 words each;
+        // for several rows of x the halves run one after the other, which
+        // bounds how many activation words the compiler keeps in flight.
+        constexpr int kHalfUnroll = (MP == 1) ? 2 : 1;
+        if constexpr (MIXED) {
+          float a0[JQ][MP], a1[JQ][MP];
 #pragma unroll
-        for (int j = 0; j < JR; ++j)
+          for (int j = 0; j < JQ; ++j)
 #pragma unroll
-          for (int m = 0; m < MP; ++m)
-            v[j * MP + m] = active ? sc[j] * ((acc[j][m].x + acc[j][m].y) -
-                                              zc[j] * (xs2[m].x + xs2[m].y))
-                                   : 0.0f;
-        half_transpose_reduce<V>(v, p);
+            for (int m = 0; m < MP; ++m) a0[j][m] = a1[j][m] = 0.0f;
+#pragma unroll kHalfUnroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint4 c[JQ];
 #pragma unroll
-        for (int i2 = 0; i2 < RM::kPerLane; ++i2) run[pass][i2] += v[i2];
+            for (int j = 0; j < JQ; ++j) {
+              const int r = warp * 16 + 4 * (pass * JQ + j) + rq;
+              c[j] = active ? *reinterpret_cast<const uint4*>(stage + r * pitch + p * 32 + hf * 16)
+                            : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              uint4 xw[MP];
+#pragma unroll
+              for (int m = 0; m < MP; ++m)
+                xw[m] = *reinterpret_cast<const uint4*>(stage + SL::kX + m * SL::kXRow +
+                                                        p * kXbChunk + 16 * (4 * hf + wd));
+#pragma unroll
+              for (int j = 0; j < JQ; ++j) {
+                const uint32_t w = wd == 0 ? c[j].x : wd == 1 ? c[j].y : wd == 2 ? c[j].z : c[j].w;
+#pragma unroll
+                for (int m = 0; m < MP; ++m) mixed_word(w, xw[m], a0[j][m], a1[j][m]);
+              }
+            }
+          }
+          // partial of (row, m) over this lane's 64 inputs:
+          //   s16 * (sum x (128 + q) - (128 + z) * sum x)
+#pragma unroll
+          for (int j = 0; j < JQ; ++j)
+#pragma unroll
+            for (int m = 0; m < MP; ++m)
+              v[j * MP + m] = active ? sc[j] * ((a0[j][m] + a1[j][m]) - (128.0f + zc[j]) * xsum[m])
+                                     : 0.0f;
+        } else {
+          float2 acc[JQ][MP];
+          float cz[JQ];
+#pragma unroll
+          for (int j = 0; j < JQ; ++j) {
+            cz[j] = -(128.0f + zc[j]);
+#pragma unroll
+            for (int m = 0; m < MP; ++m) acc[j][m] = make_float2(0.0f, 0.0f);
+          }
+#pragma unroll kHalfUnroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint4 c[JQ];
+#pragma unroll
+            for (int j = 0; j < JQ; ++j) {
+              const int r = warp * 16 + 4 * (pass * JQ + j) + rq;
+              c[j] = active ? *reinterpret_cast<const uint4*>(stage + r * pitch + p * 32 + hf * 16)
+                            : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              float2 xv[MP][4];
+#pragma unroll
+              for (int m = 0; m < MP; ++m) {
+                const float4* xp = reinterpret_cast<const float4*>(
+                    stage + SL::kX + m * SL::kXRow + p * kXfChunk + 32 * (4 * hf + wd));
+                const float4 lo = xp[0], hi = xp[1];
+                xv[m][0] = make_float2(lo.x, lo.y);
+                xv[m][1] = make_float2(lo.z, lo.w);
+                xv[m][2] = make_float2(hi.x, hi.y);
+                xv[m][3] = make_float2(hi.z, hi.w);
+              }
+#pragma unroll
+              for (int j = 0; j < JQ; ++j) {
+                const uint32_t w = wd == 0 ? c[j].x : wd == 1 ? c[j].y : wd == 2 ? c[j].z : c[j].w;
+                float2 d01, d23, d45, d67;           // exact (q - z) for the word's 8 inputs
+                widen_word(w, cz[j], d01, d23, d45, d67);
+#pragma unroll
+                for (int m = 0; m < MP; ++m) {
+                  float2 a = acc[j][m];
+                  a = __ffma2_rn(d01, xv[m][0], a);
+                  a = __ffma2_rn(d23, xv[m][1], a);
+                  a = __ffma2_rn(d45, xv[m][2], a);
+                  a = __ffma2_rn(d67, xv[m][3], a);
+                  acc[j][m] = a;
+                }
+              }
+            }
+          }
+          // partial of (row, m) over this lane's 64 inputs: s16 * sum x' (q - z)
+#pragma unroll
+          for (int j = 0; j < JQ; ++j)
+#pragma unroll
+            for (int m = 0; m < MP; ++m)
+              v[j * MP + m] = active ? sc[j] * (acc[j][m].x + acc[j][m].y) : 0.0f;
+        }
+        group_transpose_reduce<V, 8>(v, p);
+#pragma unroll
+        for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[pass][i2] += v[i2];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
@@ -325,32 +470,25 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
     const bool piece_end = (s == g.NS - 1) || (i == ntiles - 1);
     if (piece_end) {
       const bool whole = (piece_s0 == 0) && (s == g.NS - 1);
-      if (whole) {
-        if (!aborted && RM::writer(p)) {
+      if (!aborted && GM::writer(p)) {
 #pragma unroll
-          for (int pass = 0; pass < kPasses; ++pass)
+        for (int pass = 0; pass < kPasses; ++pass)
 #pragma unroll
-            for (int i2 = 0; i2 < RM::kPerLane; ++i2) {
-              const int idx = RM::index(i2, p);
-              const int j = idx / MP, m = idx % MP;
-              const int n = b * kTileRows + warp * 16 + 2 * (pass * JR + j) + h;
-              if (m < prm.M && n < g.N) prm.y[(size_t)m * g.N + n] = run[pass][i2];
-            }
-        }
-      } else {
-        // Partial piece: its slot is its first slab.
-        if (!aborted && RM::writer(p)) {
-#pragma unroll
-          for (int pass = 0; pass < kPasses; ++pass)
-#pragma unroll
-            for (int i2 = 0; i2 < RM::kPerLane; ++i2) {
-              const int idx = RM::index(i2, p);
-              const int j = idx / MP, m = idx % MP;
-              const int n = b * kTileRows + warp * 16 + 2 * (pass * JR + j) + h;
-              if (m < prm.M)
+          for (int i2 = 0; i2 < GM::kPerLane; ++i2) {
+            const int idx = GM::index(i2, p);
+            const int j = idx / MP, m = idx % MP;
+            const int n = b * kTileRows + warp * 16 + 4 * (pass * JQ + j) + rq;
+            if (m < prm.M) {
+              if (whole) {
+                if (n < g.N) prm.y[(size_t)m * g.N + n] = run[pass][i2];
+              } else {
+                // partial piece: its slot is its first slab
                 prm.partials[((size_t)piece_s0 * MP + m) * g.Npad + n] = run[pass][i2];
+              }
             }
-        }
+          }
+      }
+      if (!whole) {
         __threadfence();
         __syncwarp();
         const long long ub = (long long)b * g.NS;
@@ -382,7 +520,7 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
 #pragma unroll
       for (int a = 0; a < kPasses; ++a)
 #pragma unroll
-        for (int i2 = 0; i2 < RM::kPerLane; ++i2) run[a][i2] = 0.0f;
+        for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[a][i2] = 0.0f;
       piece_s0 = -1;
     }
   }
@@ -395,22 +533,24 @@ struct GemvConfig {
   size_t smem;
 };
 
-template <int MP, int JR, int STAGES, int MINB>
+template <int MP, int JQ, int STAGES, int MINB, bool MIXED>
 static GemvConfig gemv_config() {
   GemvConfig c;
-  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JR, STAGES, MINB>);
-  c.smem = (size_t)STAGES * StageLayout<MP>::kBytes + 2 * STAGES * sizeof(uint64_t) + 16;
+  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, MINB, MIXED>);
+  c.smem = (size_t)STAGES * StageLayout<MP, MIXED>::kBytes + 2 * STAGES * sizeof(uint64_t) + 16;
   return c;
 }
 
 static int padded_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
-static GemvConfig pick_gemv(int M) {
+// Mixed path for M <= 4 without an activation scale; packed fp32 path for the
+// AWQ fold and for M > 4 (where one widening per code is shared by 8 rows).
+static GemvConfig pick_gemv(int M, bool awq) {
   switch (padded_m(M)) {
-    case 1: return gemv_config<1, 8, 3, 2>();
-    case 2: return gemv_config<2, 4, 3, 2>();
-    case 4: return gemv_config<4, 4, 4, 1>();
-    default: return gemv_config<8, 2, 4, 1>();
+    case 1: return awq ? gemv_config<1, 4, 3, 2, false>() : gemv_config<1, 4, 3, 2, true>();
+    case 2: return awq ? gemv_config<2, 2, 4, 1, false>() : gemv_config<2, 2, 3, 2, true>();
+    case 4: return awq ? gemv_config<4, 2, 4, 1, false>() : gemv_config<4, 2, 4, 1, true>();
+    default: return gemv_config<8, 2, 4, 1, false>();
   }
 }
 
@@ -438,7 +578,7 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   prm.wait_ns = wait_ns;
   prm.drain_ns = 1000000000ull;
 
-  const GemvConfig c = pick_gemv(M);
+  const GemvConfig c = pick_gemv(M, inv_s != nullptr);
   int per_sm = 0;
   cudaError_t e = kernel_setup(c.fn, c.smem, kGemvThreads, &per_sm);
   if (e != cudaSuccess) return e;

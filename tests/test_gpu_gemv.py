@@ -24,7 +24,19 @@ def test_gemv_small_all_m(N, K, sym):
         check_close(y, yref, f"N={N} K={K} M={M}")
 
 
-@pytest.mark.parametrize("M", [1, 4, 8])
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_row_tile_split_across_many_ctas(M):
+    """N = 128 with K = 28672: one row tile of 56 slabs, more CTAs than a row
+    tile has slabs, so every CTA holds a piece and the last one adds them."""
+    N, K = 128, 28672
+    W = inputs.weights(N, K, 0.015, seed=7)
+    qw, P, s, z = quantize_and_check(W, None, False)
+    x = inputs.activations(M, K, seed=8)
+    y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+    check_close(y, oracle.linear(x, P, s, z, K, sym=False))
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
 def test_gemv_awq_fold_small(M):
     N, K = 256, 1536
     W = inputs.weights(N, K, 0.015, seed=91)
