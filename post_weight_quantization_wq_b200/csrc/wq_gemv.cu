@@ -19,15 +19,16 @@
 //     prepares the tile's activation slab once for the whole CTA: bf16 x plus
 //     fp32 sums of x per 64 inputs (mixed path), or fp32 x * (1/s) (packed
 //     path); eight consumer warps compute;
-//   * dequantization in registers: the nibbles at bits 4i and 16+4i of a word,
-//     masked and OR-ed into 0x43004300, are two bf16 values 128 + q (one LOP3
-//     for two codes, exact).  Mixed path (no activation scale, M <= 4): the
-//     bf16 codes meet the bf16 activations in sm_100's mixed-precision FMA
-//     (bf16 x bf16 + fp32, exact product), and each (row, group) sum is
-//     corrected by (128 + z) * sum(x) and scaled by the fp16 scale in fp32.
-//     Packed path (AWQ fold, M = 8): each 128 + q is widened to the fp32 code
-//     q - z by a mixed-precision add, and packed fp32x2 FMAs multiply it with
-//     the fp32 activations;
+//   * dequantization in registers, two codes per LOP3 (no conversion
+//     instruction): mixed path (no activation scale, M <= 4): masked nibble
+//     pairs OR-ed into fp16 exponent patterns are 1024 + q or 64 + q exactly
+//     (4 LOP3 + 1 shift per 8 codes); the producer gives each 64-input chunk
+//     of x an exact power-of-two scale into fp16; sm_100's mixed-precision FMA
+//     (fp16 x fp16 + fp32, exact product) accumulates, and each (row, chunk)
+//     sum loses the bias terms and z * sum(x) and is scaled by s16 * 2^-e in
+//     fp32.  Packed path (AWQ fold, M = 8): bf16 pairs 128 + q (mask into
+//     0x43004300) are widened to the fp32 code q - z by a mixed-precision add
+//     and packed fp32x2 FMAs multiply them with the fp32 activations;
 //   * 8 lanes share a row of a tile, lane p covering inputs 64p..64p+63 of
 //     the slab; their partial sums of several rows are combined with a
 //     transposing shuffle reduction;
@@ -39,6 +40,8 @@
 //   * every wait is bounded (globaltimer): on timeout the kernel records the
 //     device error word, stops issuing copies, waits (bounded) for its copies
 //     in flight and returns.
+#include <type_traits>
+
 #include "wq_common.cuh"
 
 namespace wq {
@@ -56,6 +59,9 @@ struct GemvParams {
   long long tiles;         // NS * NB
   unsigned long long wait_ns;
   unsigned long long drain_ns;
+  // Masks and exponent patterns of the code extraction, passed at run time so
+  // that each extraction is one 3-register LOP3 instead of two immediate ops.
+  uint32_t lop_mask_lo, lop_mask_hi, lop_f16_1024, lop_f16_64, lop_bf16_128;
 };
 
 constexpr int kConsumerWarps = 8;
@@ -70,8 +76,11 @@ template <int MP, bool MIXED>
 struct StageLayout {
   static constexpr int kX = kMaxFullTile;
   static constexpr int kXRow = kChunks * (MIXED ? kXbChunk : kXfChunk);
-  static constexpr int kXsum = kX + MP * kXRow;                       // fp32 [MP][8]
-  static constexpr int kBytes = kXsum + (MIXED ? MP * kChunks * 4 : 0);
+  static constexpr int kXsum = kX + MP * kXRow;     // mixed: float4 [MP][8] chunk info
+  static constexpr int kBytes = kXsum + (MIXED ? MP * kChunks * 16 : 0);
+  // raw activation slot: bf16 [MP][512], then fp32 [512] of the AWQ factor
+  static constexpr int kRawInv = MP * kSlabK * 2;
+  static constexpr int kRawBytes = kRawInv + (MIXED ? 0 : kSlabK * 4);
 };
 
 // Sum v[] over the L lanes (L = 8 or 16, lane index p) of a lane group.
@@ -109,37 +118,57 @@ struct GroupMap {
   __device__ static int index(int i, int p) { return V >= L ? i + kPerLane * p : (p >> kShift); }
 };
 
-// Two bf16 values 128 + q of the nibbles at bits [4i, 4i+4) and [16+4i, 20+4i)
-// of w (exact: 128..143 are bf16 integers).
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) {
-  return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+// (a & b) | c in one LOP3 with all three operands in registers.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
-// acc += x_k * (128 + q_k) for the 8 inputs of one word, with sm_100's
-// mixed-precision FMA (bf16 * bf16 + fp32, one rounding, exact product).
-// xw holds the 8 bf16 activations as pairs (x0,x1) (x2,x3) (x4,x5) (x6,x7).
-__device__ __forceinline__ void mixed_word(uint32_t w, const uint4& xw, float& a0, float& a1) {
-  const uint32_t v0 = nib_pair(w, 0), v1 = nib_pair(w, 1), v2 = nib_pair(w, 2),
-                 v3 = nib_pair(w, 3);   // vi = (q_i, q_{i+4})
-  asm("{\n\t.reg .b16 q0, q4, q1, q5, q2, q6, q3, q7, x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
-      "mov.b32 {q0, q4}, %2;\n\tmov.b32 {q1, q5}, %3;\n\t"
-      "mov.b32 {q2, q6}, %4;\n\tmov.b32 {q3, q7}, %5;\n\t"
-      "mov.b32 {x0, x1}, %6;\n\tmov.b32 {x2, x3}, %7;\n\t"
-      "mov.b32 {x4, x5}, %8;\n\tmov.b32 {x6, x7}, %9;\n\t"
-      "fma.rn.f32.bf16 %0, q0, x0, %0;\n\tfma.rn.f32.bf16 %1, q1, x1, %1;\n\t"
-      "fma.rn.f32.bf16 %0, q2, x2, %0;\n\tfma.rn.f32.bf16 %1, q3, x3, %1;\n\t"
-      "fma.rn.f32.bf16 %0, q4, x4, %0;\n\tfma.rn.f32.bf16 %1, q5, x5, %1;\n\t"
-      "fma.rn.f32.bf16 %0, q6, x6, %0;\n\tfma.rn.f32.bf16 %1, q7, x7, %1;\n\t}"
+struct LopConsts {
+  uint32_t mlo, mhi, f1024, f64, b128;   // 0x000F000F 0x00F000F0 0x64006400 0x54005400 0x43004300
+};
+
+// Two bf16 values 128 + q of the nibbles at bits [4i, 4i+4) and [16+4i, 20+4i)
+// of w (exact: 128..143 are bf16 integers).
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i, const LopConsts& k) {
+  return and_or(w >> (4 * i), k.mlo, k.b128);
+}
+
+// acc += x_k * c_k for the 8 inputs of one word, with sm_100's mixed-precision
+// FMA (fp16 * fp16 + fp32, one rounding, exact product).  The codes come out
+// of 4 LOP3s as fp16 pairs: OR-ing the nibbles at bits [0,4) / [16,20) into
+// 0x6400 (1024, unit step) gives 1024 + q; OR-ing the nibbles at bits [4,8) /
+// [20,24) into 0x5400 (64, step 1/16 per mantissa bit, so 1 per nibble unit)
+// gives 64 + q; the same again on w >> 8 for the other four.  xw holds the
+// activations as fp16 pairs (x0,x4) (x1,x5) (x2,x6) (x3,x7), so
+//   a0 + a1 = sum_k x_k q_k + 1024 (x0+x2+x4+x6) + 64 (x1+x3+x5+x7).
+__device__ __forceinline__ void mixed_word(uint32_t w, const uint4& xw, float& a0, float& a1,
+                                           const LopConsts& k) {
+  const uint32_t w8 = w >> 8;
+  const uint32_t ca = and_or(w, k.mlo, k.f1024);     // (1024 + q0, 1024 + q4)
+  const uint32_t cb = and_or(w, k.mhi, k.f64);       // (64 + q1, 64 + q5)
+  const uint32_t cc = and_or(w8, k.mlo, k.f1024);    // (1024 + q2, 1024 + q6)
+  const uint32_t cd = and_or(w8, k.mhi, k.f64);      // (64 + q3, 64 + q7)
+  asm("{\n\t.reg .b16 c0, c4, c1, c5, c2, c6, c3, c7, x0, x4, x1, x5, x2, x6, x3, x7;\n\t"
+      "mov.b32 {c0, c4}, %2;\n\tmov.b32 {c1, c5}, %3;\n\t"
+      "mov.b32 {c2, c6}, %4;\n\tmov.b32 {c3, c7}, %5;\n\t"
+      "mov.b32 {x0, x4}, %6;\n\tmov.b32 {x1, x5}, %7;\n\t"
+      "mov.b32 {x2, x6}, %8;\n\tmov.b32 {x3, x7}, %9;\n\t"
+      "fma.rn.f32.f16 %0, c0, x0, %0;\n\tfma.rn.f32.f16 %1, c4, x4, %1;\n\t"
+      "fma.rn.f32.f16 %0, c1, x1, %0;\n\tfma.rn.f32.f16 %1, c5, x5, %1;\n\t"
+      "fma.rn.f32.f16 %0, c2, x2, %0;\n\tfma.rn.f32.f16 %1, c6, x6, %1;\n\t"
+      "fma.rn.f32.f16 %0, c3, x3, %0;\n\tfma.rn.f32.f16 %1, c7, x7, %1;\n\t}"
       : "+f"(a0), "+f"(a1)
-      : "r"(v0), "r"(v1), "r"(v2), "r"(v3), "r"(xw.x), "r"(xw.y), "r"(xw.z), "r"(xw.w));
+      : "r"(ca), "r"(cb), "r"(cc), "r"(cd), "r"(xw.x), "r"(xw.y), "r"(xw.z), "r"(xw.w));
 }
 
 // The 8 codes of one word as exact fp32 (q - z) pairs, in input order:
 // f32(128 + q) + cz with cz = -(128 + z), by the mixed-precision add.
 __device__ __forceinline__ void widen_word(uint32_t w, float cz, float2& d01, float2& d23,
-                                           float2& d45, float2& d67) {
-  const uint32_t v0 = nib_pair(w, 0), v1 = nib_pair(w, 1), v2 = nib_pair(w, 2),
-                 v3 = nib_pair(w, 3);
+                                           float2& d45, float2& d67, const LopConsts& k) {
+  const uint32_t v0 = nib_pair(w, 0, k), v1 = nib_pair(w, 1, k), v2 = nib_pair(w, 2, k),
+                 v3 = nib_pair(w, 3, k);
   asm("{\n\t.reg .b16 q0, q4, q1, q5, q2, q6, q3, q7;\n\t"
       "mov.b32 {q0, q4}, %8;\n\tmov.b32 {q1, q5}, %9;\n\t"
       "mov.b32 {q2, q6}, %10;\n\tmov.b32 {q3, q7}, %11;\n\t"
@@ -169,26 +198,28 @@ struct XSlice {
   float4 inv[MIXED ? 1 : 4];
 };
 
+// Read lane l's share (inputs 16l .. 16l+15 of the slab) from a raw slot.
 template <int MP, bool MIXED>
-__device__ __forceinline__ void load_x_slice(XSlice<MP, MIXED>& xs, const GemvParams& prm, int s,
-                                             int lane) {
-  const int k = s * kSlabK + 16 * lane;
-  const bool ok = k < prm.g.K;
+__device__ __forceinline__ void read_x_slice(XSlice<MP, MIXED>& xs, const uint8_t* raw,
+                                             const GemvParams& prm, int s, int lane) {
+  using SL = StageLayout<MP, MIXED>;
+  const bool ok = s * kSlabK + 16 * lane < prm.g.K;   // inside the slab's groups
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
     xs.xb[m][0] = make_uint4(0, 0, 0, 0);
     xs.xb[m][1] = make_uint4(0, 0, 0, 0);
     if (ok && m < prm.M) {
-      const uint4* src = reinterpret_cast<const uint4*>(prm.x + (size_t)m * prm.g.K + k);
-      xs.xb[m][0] = __ldg(src);
-      xs.xb[m][1] = __ldg(src + 1);
+      const uint4* src = reinterpret_cast<const uint4*>(raw + m * kSlabK * 2 + 32 * lane);
+      xs.xb[m][0] = src[0];
+      xs.xb[m][1] = src[1];
     }
   }
   if constexpr (!MIXED) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       xs.inv[q] = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (ok && prm.inv_s) xs.inv[q] = __ldg(reinterpret_cast<const float4*>(prm.inv_s + k) + q);
+      if (ok && prm.inv_s)
+        xs.inv[q] = reinterpret_cast<const float4*>(raw + SL::kRawInv + 64 * lane)[q];
     }
   }
 }
@@ -204,15 +235,48 @@ __device__ __forceinline__ void store_x_slice(const XSlice<MP, MIXED>& xs, uint8
     const uint32_t r[8] = {xs.xb[m][0].x, xs.xb[m][0].y, xs.xb[m][0].z, xs.xb[m][0].w,
                            xs.xb[m][1].x, xs.xb[m][1].y, xs.xb[m][1].z, xs.xb[m][1].w};
     if constexpr (MIXED) {
-      uint4* dst = reinterpret_cast<uint4*>(stage + SL::kX + m * SL::kXRow + c * kXbChunk + sub * 32);
-      dst[0] = xs.xb[m][0];
-      dst[1] = xs.xb[m][1];
-      float sum = 0.0f;
+      // fp16 copy of the chunk scaled by 2^e, e chosen from the chunk's largest
+      // |x| so that it lands in [2^14, 2^15): bf16's 8-bit significands fit
+      // fp16's 11 bits, so every value within 2^-28 of the largest is exact.
+      float xf[16];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) sum += bf16_lo(r[q]) + bf16_hi(r[q]);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-      if (sub == 0) reinterpret_cast<float*>(stage + SL::kXsum)[m * kChunks + c] = sum;
+      for (int q = 0; q < 8; ++q) {
+        xf[2 * q] = bf16_lo(r[q]);
+        xf[2 * q + 1] = bf16_hi(r[q]);
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(xf[q]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+      const int eb = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+      int e = (eb == 0) ? 0 : 141 - eb;            // amax * 2^e in [2^14, 2^15)
+      e = e < -126 ? -126 : (e > 126 ? 126 : e);
+      const float scale = __uint_as_float((uint32_t)(e + 127) << 23);
+      const float unscale = __uint_as_float((uint32_t)(127 - e) << 23);
+      uint32_t hw[8];
+      float sa = 0.0f, sb = 0.0f;                 // sums at the 1024- and 64-biased slots
+#pragma unroll
+      for (int wd = 0; wd < 2; ++wd) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __half lo = __float2half_rn(__fmul_rn(xf[8 * wd + i], scale));
+          const __half hi = __float2half_rn(__fmul_rn(xf[8 * wd + i + 4], scale));
+          hw[4 * wd + i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+          const float f = __half2float(lo) + __half2float(hi);
+          if (i & 1) sb += f; else sa += f;
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(stage + SL::kX + m * SL::kXRow + c * kXbChunk + sub * 32);
+      dst[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      dst[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+      sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
+      sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 2);
+      sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
+      sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 2);
+      if (sub == 0)
+        reinterpret_cast<float4*>(stage + SL::kXsum)[m * kChunks + c] =
+            make_float4(1024.0f * sa + 64.0f * sb, sa + sb, unscale, 0.0f);
     } else {
       float4* dst = reinterpret_cast<float4*>(stage + SL::kX + m * SL::kXRow + c * kXfChunk + sub * 64);
 #pragma unroll
@@ -226,14 +290,16 @@ __device__ __forceinline__ void store_x_slice(const XSlice<MP, MIXED>& xs, uint8
   }
 }
 
-template <int MP, int JQ, int STAGES, int MINB, bool MIXED>
+template <int MP, int JQ, int STAGES, int RAWS, int MINB, bool MIXED>
 __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvParams prm) {
   using SL = StageLayout<MP, MIXED>;
   extern __shared__ __align__(128) uint8_t smem[];
   const Geom g = prm.g;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * SL::kBytes);
+  uint8_t* raw_ring = smem + STAGES * SL::kBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(raw_ring + RAWS * SL::kRawBytes);
   uint64_t* empty_bar = full_bar + STAGES;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty_bar + STAGES);
+  uint64_t* raw_bar = empty_bar + STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(raw_bar + RAWS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -247,6 +313,7 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
       mbar_init(&full_bar[i], 1 + 32);           // producer's expect_tx + its 32 lanes
       mbar_init(&empty_bar[i], kConsumerWarps);
     }
+    for (int i = 0; i < RAWS; ++i) mbar_init(&raw_bar[i], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -258,13 +325,35 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
 
   if (warp == kConsumerWarps) {
     // ---------------------------------------------------------------- producer
-    int issued = 0;
-    XSlice<MP, MIXED> xs;
-    if (ntiles > 0) load_x_slice<MP, MIXED>(xs, prm, (int)(t0 % g.NS), lane);
+    // The raw activation slab (and AWQ factor) of tile i is bulk-copied into
+    // raw slot i % RAWS, RAWS tiles ahead of its use, so the slab is already
+    // in shared memory when the producer converts it into tile i's stage.
+    int issued = 0, raw_issued = 0;
+    int pb = (int)(t0 / g.NS), ps = (int)(t0 % g.NS), pf = ps;
+    auto next_slab = [&](int v) { return v + 1 == g.NS ? 0 : v + 1; };
+    auto issue_raw = [&](int slot, int slab) {       // lane 0 only
+      uint8_t* dst = raw_ring + slot * SL::kRawBytes;
+      const int gsx = slab_groups(g, slab);
+      const uint32_t xb = gsx * kGroup * 2, ib = prm.inv_s ? gsx * kGroup * 4 : 0;
+      mbar_arrive_expect_tx(&raw_bar[slot], prm.M * xb + ib);
+      for (int m = 0; m < prm.M; ++m)
+        bulk_copy_g2s(dst + m * kSlabK * 2, prm.x + (size_t)m * g.K + slab * kSlabK, xb,
+                      &raw_bar[slot]);
+      if (ib) bulk_copy_g2s(dst + SL::kRawInv, prm.inv_s + slab * kSlabK, ib, &raw_bar[slot]);
+    };
+    if (lane == 0)
+      for (int r = 0; r < RAWS && r < ntiles; ++r) {
+        issue_raw(r, pf);
+        pf = next_slab(pf);
+      }
+    raw_issued = ntiles < RAWS ? ntiles : RAWS;
+    pf = __shfl_sync(0xFFFFFFFFu, pf, 0);
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % STAGES;
+      const int rs = i % RAWS;
       bool ok = true;
       if (i >= STAGES) ok = mbar_wait_bounded(&empty_bar[st], ((i / STAGES) - 1) & 1, prm.wait_ns);
+      if (ok) ok = mbar_wait_bounded(&raw_bar[rs], (i / RAWS) & 1, prm.wait_ns);
       ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
       if (!ok) {
         if (lane == 0) {
@@ -273,24 +362,38 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
         }
         break;
       }
-      const long long u = t0 + i;
-      const int b = (int)(u / g.NS), s = (int)(u % g.NS);
       uint8_t* stage = smem + st * SL::kBytes;
       if (lane == 0) {
-        const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, s));
+        const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, ps));
         mbar_arrive_expect_tx(&full_bar[st], tbytes);
-        bulk_copy_g2s(stage, prm.packed + tile_offset(g, s, b), tbytes, &full_bar[st]);
+        bulk_copy_g2s(stage, prm.packed + tile_offset(g, ps, pb), tbytes, &full_bar[st]);
       }
+      XSlice<MP, MIXED> xs;
+      read_x_slice<MP, MIXED>(xs, raw_ring + rs * SL::kRawBytes, prm, ps, lane);
       store_x_slice<MP, MIXED>(xs, stage, prm, lane);
       mbar_arrive(&full_bar[st]);
       issued = i + 1;
-      if (i + 1 < ntiles) load_x_slice<MP, MIXED>(xs, prm, (int)((u + 1) % g.NS), lane);
+      ps = next_slab(ps);
+      if (ps == 0) ++pb;
+      __syncwarp();                      // every lane has read raw slot rs
+      if (i + RAWS < ntiles) {
+        if (lane == 0) {
+          fence_proxy_async_shared();    // generic reads before the async overwrite
+          issue_raw(rs, pf);
+        }
+        pf = next_slab(pf);
+        ++raw_issued;
+      }
     }
     if (lane == 0 && *abort_flag) {
       // Wait (bounded) for every copy still in flight before the CTA exits.
       for (int st = 0; st < STAGES && st < issued; ++st) {
         const int uses = (issued - 1 - st) / STAGES + 1;   // copies issued on stage st
         mbar_wait_bounded(&full_bar[st], (uses - 1) & 1, prm.drain_ns);
+      }
+      for (int r = 0; r < RAWS && r < raw_issued; ++r) {
+        const int uses = (raw_issued - 1 - r) / RAWS + 1;
+        mbar_wait_bounded(&raw_bar[r], (uses - 1) & 1, prm.drain_ns);
       }
     }
     return;
@@ -302,6 +405,8 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
   constexpr int V = JQ * MP;
   constexpr int kPasses = 4 / JQ;
   using GM = GroupMap<V, 8>;
+  const LopConsts lk{prm.lop_mask_lo, prm.lop_mask_hi, prm.lop_f16_1024, prm.lop_f16_64,
+                     prm.lop_bf16_128};
 
   float run[kPasses][GM::kPerLane];
 #pragma unroll
@@ -310,10 +415,10 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
     for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[a][i2] = 0.0f;
   int piece_s0 = -1;                // first slab of the current row tile in this CTA
   bool aborted = false;
+  int b = (int)(t0 / g.NS), s = (int)(t0 % g.NS) - 1;
 
   for (int i = 0; i < ntiles; ++i) {
-    const long long u = t0 + i;
-    const int b = (int)(u / g.NS), s = (int)(u % g.NS);
+    if (++s == g.NS) { s = 0; ++b; }
     const int gs = slab_groups(g, s);
     const int st = i % STAGES;
     if (piece_s0 < 0) piece_s0 = s;
@@ -332,13 +437,17 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
       const uint8_t* stage = smem + st * SL::kBytes;
       const uint8_t* meta = stage + kTileRows * gs * kCodeBytesPerGroupRow;
       const int pitch = gs * kCodeBytesPerGroupRow;
-      const bool active = p < 2 * gs;
       const int grp = p >> 1;
-      float xsum[MP];
+      // Full slabs (all but possibly the last) take a predicate-free copy of
+      // the compute; in a ragged last slab lanes past its groups sit out.
+      auto tile_compute = [&](auto ragged_tag) {
+      constexpr bool kRagged = decltype(ragged_tag)::value;
+      const bool active = !kRagged || p < 2 * gs;
+      float4 xinfo[MIXED ? MP : 1];    // mixed: (bias, sum x, 2^-e, -) of this lane's chunk
       if constexpr (MIXED) {
 #pragma unroll
         for (int m = 0; m < MP; ++m)
-          xsum[m] = reinterpret_cast<const float*>(stage + SL::kXsum)[m * kChunks + p];
+          xinfo[m] = reinterpret_cast<const float4*>(stage + SL::kXsum)[m * kChunks + p];
       }
 
 #pragma unroll 1
@@ -391,17 +500,18 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
               for (int j = 0; j < JQ; ++j) {
                 const uint32_t w = wd == 0 ? c[j].x : wd == 1 ? c[j].y : wd == 2 ? c[j].z : c[j].w;
 #pragma unroll
-                for (int m = 0; m < MP; ++m) mixed_word(w, xw[m], a0[j][m], a1[j][m]);
+                for (int m = 0; m < MP; ++m) mixed_word(w, xw[m], a0[j][m], a1[j][m], lk);
               }
             }
           }
           // partial of (row, m) over this lane's 64 inputs:
-          //   s16 * (sum x (128 + q) - (128 + z) * sum x)
+          //   s16 * 2^-e * ((acc - bias) - z * sum x)
 #pragma unroll
           for (int j = 0; j < JQ; ++j)
 #pragma unroll
             for (int m = 0; m < MP; ++m)
-              v[j * MP + m] = active ? sc[j] * ((a0[j][m] + a1[j][m]) - (128.0f + zc[j]) * xsum[m])
+              v[j * MP + m] = active ? (sc[j] * xinfo[m].z) *
+                                           (((a0[j][m] + a1[j][m]) - xinfo[m].x) - zc[j] * xinfo[m].y)
                                      : 0.0f;
         } else {
           float2 acc[JQ][MP];
@@ -438,7 +548,7 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
               for (int j = 0; j < JQ; ++j) {
                 const uint32_t w = wd == 0 ? c[j].x : wd == 1 ? c[j].y : wd == 2 ? c[j].z : c[j].w;
                 float2 d01, d23, d45, d67;           // exact (q - z) for the word's 8 inputs
-                widen_word(w, cz[j], d01, d23, d45, d67);
+                widen_word(w, cz[j], d01, d23, d45, d67, lk);
 #pragma unroll
                 for (int m = 0; m < MP; ++m) {
                   float2 a = acc[j][m];
@@ -462,6 +572,9 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
 #pragma unroll
         for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[pass][i2] += v[i2];
       }
+      };
+      if (gs == kSlabGroups) tile_compute(std::false_type{});
+      else tile_compute(std::true_type{});
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
@@ -533,11 +646,13 @@ struct GemvConfig {
   size_t smem;
 };
 
-template <int MP, int JQ, int STAGES, int MINB, bool MIXED>
+template <int MP, int JQ, int STAGES, int RAWS, int MINB, bool MIXED>
 static GemvConfig gemv_config() {
+  using SL = StageLayout<MP, MIXED>;
   GemvConfig c;
-  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, MINB, MIXED>);
-  c.smem = (size_t)STAGES * StageLayout<MP, MIXED>::kBytes + 2 * STAGES * sizeof(uint64_t) + 16;
+  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, RAWS, MINB, MIXED>);
+  c.smem = (size_t)STAGES * SL::kBytes + (size_t)RAWS * SL::kRawBytes +
+           (2 * STAGES + RAWS) * sizeof(uint64_t) + 16;
   return c;
 }
 
@@ -545,12 +660,13 @@ static int padded_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
 // Mixed path for M <= 4 without an activation scale; packed fp32 path for the
 // AWQ fold and for M > 4 (where one widening per code is shared by 8 rows).
+// Stage counts keep two CTAs per SM where M <= 2.
 static GemvConfig pick_gemv(int M, bool awq) {
   switch (padded_m(M)) {
-    case 1: return awq ? gemv_config<1, 4, 3, 2, false>() : gemv_config<1, 4, 3, 2, true>();
-    case 2: return awq ? gemv_config<2, 2, 4, 1, false>() : gemv_config<2, 2, 3, 2, true>();
-    case 4: return awq ? gemv_config<4, 2, 4, 1, false>() : gemv_config<4, 2, 4, 1, true>();
-    default: return gemv_config<8, 2, 4, 1, false>();
+    case 1: return awq ? gemv_config<1, 4, 2, 2, 2, false>() : gemv_config<1, 4, 2, 3, 3, true>();
+    case 2: return awq ? gemv_config<2, 2, 4, 2, 1, false>() : gemv_config<2, 2, 2, 4, 2, true>();
+    case 4: return awq ? gemv_config<4, 2, 4, 2, 1, false>() : gemv_config<4, 2, 4, 3, 1, true>();
+    default: return gemv_config<8, 2, 3, 2, 1, false>();
   }
 }
 
@@ -577,6 +693,11 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   prm.tiles = (long long)prm.g.NS * prm.g.NB;
   prm.wait_ns = wait_ns;
   prm.drain_ns = 1000000000ull;
+  prm.lop_mask_lo = 0x000F000Fu;
+  prm.lop_mask_hi = 0x00F000F0u;
+  prm.lop_f16_1024 = 0x64006400u;
+  prm.lop_f16_64 = 0x54005400u;
+  prm.lop_bf16_128 = 0x43004300u;
 
   const GemvConfig c = pick_gemv(M, inv_s != nullptr);
   int per_sm = 0;
