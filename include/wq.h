@@ -117,11 +117,14 @@ wq_status wq_quantize_rtn(const void* W, const float* awq_scale, int N, int K, i
  * Tiles are stored slab by slab and, within a slab, row-tile by row-tile;
  * every full tile has the same size, so tile (s, b) starts at
  * s * NB * full_tile + b * tile_bytes(s) with NB = ceil(N/128).  A tile holds
- * first the codes (row r: its canonical qweight words for the slab's gs
- * groups, gs*64 bytes at offset r*gs*64), then the metadata (entry (r, g) at
- * offset 128*gs*64 + (r*gs + g) * mb): mb = 2, the fp16 scale, when
- * symmetric; mb = 4, the fp16 scale in the low and the fp16 zero in the high
- * half of a little-endian uint32, when asymmetric.  Rows past N are zero.
+ * first the codes (row r: its qweight words for the slab's gs groups, gs*64
+ * bytes at offset r*gs*64), then the metadata (entry (r, g) at offset
+ * 128*gs*64 + (r*gs + g) * mb): mb = 2, the fp16 scale, when symmetric;
+ * mb = 4, the fp16 scale in the low and the fp16 zero in the high half of a
+ * little-endian uint32, when asymmetric.  Each code word is the canonical
+ * word with its nibbles interleaved: nibble slot t holds canonical nibble 2t
+ * (t < 4) or 2(t-4)+1 (t >= 4), so one mask 0x000F000F after a shift by 4t
+ * isolates the adjacent inputs 2t and 2t+1.  Rows past N are zero.
  */
 size_t wq_packed_bytes(int N, int K, int group_size, int symmetric, int layout);
 

@@ -67,6 +67,7 @@ def _load():
             "or_linear": (None, [P, P, I, P, P, P, I, I, I, C, P, I, P, P]),
             "or_layout_bytes": (I, [I, I, C]),
             "or_relayout": (None, [P, P, P, I, I, C, P]),
+            "or_interleave_word": (ctypes.c_uint32, [ctypes.c_uint32]),
             "or_f16_selfcheck": (I, [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64]),
         }
         for name, (res, args) in sig.items():
@@ -213,6 +214,12 @@ def linear(x_bits, P, s16, z16, K: int, group: int = GROUP, sym: bool = False,
 
 def layout_bytes(N: int, K: int, sym: bool) -> int:
     return int(_load().or_layout_bytes(N, K, int(sym)))
+
+
+def interleave_word(w: int) -> int:
+    """Nibble slot t of the result holds canonical nibble 2t (t < 4) or
+    2(t-4)+1 (t >= 4)."""
+    return int(_load().or_interleave_word(int(w)))
 
 
 def relayout(P, s16, z16, N: int, K: int, sym: bool) -> np.ndarray:

@@ -339,12 +339,25 @@ void or_linear(const uint16_t* x, const float* awq_s, int64_t M,
 /* produce.  A tile holds 128 rows x one K-slab of 4 groups (512 inputs;   */
 /* the last slab may hold fewer groups).  Tiles are stored slab by slab,   */
 /* row-tile by row-tile.  Inside a tile: first the codes, row r taking     */
-/* gs*64 bytes (the row's canonical words for the slab's groups, in        */
-/* order), then the metadata, entry (r, g) at (r*gs + g) * meta bytes:     */
-/* symmetric: the fp16 scale (2 bytes); asymmetric: the fp16 scale in the  */
-/* low half and the fp16 zero in the high half of a little-endian uint32.  */
+/* gs*64 bytes (the row's words for the slab's groups, in order), then the */
+/* metadata, entry (r, g) at (r*gs + g) * meta bytes: symmetric: the fp16  */
+/* scale (2 bytes); asymmetric: the fp16 scale in the low half and the     */
+/* fp16 zero in the high half of a little-endian uint32.  Each code word   */
+/* is the canonical word with its nibbles interleaved: nibble slot t       */
+/* (bits [4t, 4t+4)) holds canonical nibble 2t for t < 4 and 2(t-4)+1 for  */
+/* t >= 4, so slots t and t+4 hold the adjacent inputs 2t and 2t+1.        */
 /* Rows N..ceil(N/128)*128-1 are padding and hold zero bytes.              */
 /* ------------------------------------------------------------------ */
+
+uint32_t or_interleave_word(uint32_t w)
+{
+    uint32_t out = 0;
+    for (int t = 0; t < 8; t++) {
+        int src = (t < 4) ? 2 * t : 2 * (t - 4) + 1;
+        out |= ((w >> (4 * src)) & 0xFu) << (4 * t);
+    }
+    return out;
+}
 
 #define OR_TILE_ROWS 128
 #define OR_SLAB_GROUPS 4
@@ -386,7 +399,8 @@ void or_relayout(const uint32_t* P, const uint16_t* s16, const uint16_t* z16,
                 for (int64_t g = 0; g < gs; g++) {
                     int64_t gg = OR_SLAB_GROUPS * s + g;
                     for (int64_t w = 0; w < 16; w++)
-                        put_u32(base + r * gs * 64 + g * 64 + w * 4, P[n * (K / 8) + gg * 16 + w]);
+                        put_u32(base + r * gs * 64 + g * 64 + w * 4,
+                                or_interleave_word(P[n * (K / 8) + gg * 16 + w]));
                     uint8_t* mp = mbase + (r * gs + g) * meta;
                     if (sym) put_u16(mp, s16[n * NG + gg]);
                     else put_u32(mp, (uint32_t)s16[n * NG + gg] | ((uint32_t)z16[n * NG + gg] << 16));

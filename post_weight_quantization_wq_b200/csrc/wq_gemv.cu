@@ -129,49 +129,52 @@ struct LopConsts {
   uint32_t mlo, mhi, f1024, f64, b128;   // 0x000F000F 0x00F000F0 0x64006400 0x54005400 0x43004300
 };
 
-// Two bf16 values 128 + q of the nibbles at bits [4i, 4i+4) and [16+4i, 20+4i)
-// of w (exact: 128..143 are bf16 integers).
+// Two bf16 values 128 + q of the nibble slots at bits [4i, 4i+4) and
+// [16+4i, 20+4i) of w, i.e. inputs 2i and 2i+1 of an interleaved word (exact:
+// 128..143 are bf16 integers).
 __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i, const LopConsts& k) {
   return and_or(w >> (4 * i), k.mlo, k.b128);
 }
 
-// acc += x_k * c_k for the 8 inputs of one word, with sm_100's mixed-precision
-// FMA (fp16 * fp16 + fp32, one rounding, exact product).  The codes come out
-// of 4 LOP3s as fp16 pairs: OR-ing the nibbles at bits [0,4) / [16,20) into
-// 0x6400 (1024, unit step) gives 1024 + q; OR-ing the nibbles at bits [4,8) /
-// [20,24) into 0x5400 (64, step 1/16 per mantissa bit, so 1 per nibble unit)
-// gives 64 + q; the same again on w >> 8 for the other four.  xw holds the
-// activations as fp16 pairs (x0,x4) (x1,x5) (x2,x6) (x3,x7), so
-//   a0 + a1 = sum_k x_k q_k + 1024 (x0+x2+x4+x6) + 64 (x1+x3+x5+x7).
+// acc += x_k * c_k for the 8 inputs of one (interleaved) word, with sm_100's
+// mixed-precision FMA (fp16 * fp16 + fp32, one rounding, exact product).  The
+// codes come out of 4 LOP3s as fp16 pairs of adjacent inputs: OR-ing the
+// nibble slots at bits [0,4) / [16,20) into 0x6400 (1024, unit step) gives
+// 1024 + q for inputs 0, 1; OR-ing the slots at bits [4,8) / [20,24) into
+// 0x5400 (64, step 1/16 per mantissa bit, so 1 per nibble unit) gives 64 + q
+// for inputs 2, 3; the same on w >> 8 for inputs 4, 5 and 6, 7.  xw holds the
+// activations as fp16 pairs (x0,x1) (x2,x3) (x4,x5) (x6,x7), so
+//   a0 + a1 = sum_k x_k q_k + 1024 (x0+x1+x4+x5) + 64 (x2+x3+x6+x7).
 __device__ __forceinline__ void mixed_word(uint32_t w, const uint4& xw, float& a0, float& a1,
                                            const LopConsts& k) {
   const uint32_t w8 = w >> 8;
-  const uint32_t ca = and_or(w, k.mlo, k.f1024);     // (1024 + q0, 1024 + q4)
-  const uint32_t cb = and_or(w, k.mhi, k.f64);       // (64 + q1, 64 + q5)
-  const uint32_t cc = and_or(w8, k.mlo, k.f1024);    // (1024 + q2, 1024 + q6)
-  const uint32_t cd = and_or(w8, k.mhi, k.f64);      // (64 + q3, 64 + q7)
-  asm("{\n\t.reg .b16 c0, c4, c1, c5, c2, c6, c3, c7, x0, x4, x1, x5, x2, x6, x3, x7;\n\t"
-      "mov.b32 {c0, c4}, %2;\n\tmov.b32 {c1, c5}, %3;\n\t"
-      "mov.b32 {c2, c6}, %4;\n\tmov.b32 {c3, c7}, %5;\n\t"
-      "mov.b32 {x0, x4}, %6;\n\tmov.b32 {x1, x5}, %7;\n\t"
-      "mov.b32 {x2, x6}, %8;\n\tmov.b32 {x3, x7}, %9;\n\t"
-      "fma.rn.f32.f16 %0, c0, x0, %0;\n\tfma.rn.f32.f16 %1, c4, x4, %1;\n\t"
-      "fma.rn.f32.f16 %0, c1, x1, %0;\n\tfma.rn.f32.f16 %1, c5, x5, %1;\n\t"
-      "fma.rn.f32.f16 %0, c2, x2, %0;\n\tfma.rn.f32.f16 %1, c6, x6, %1;\n\t"
-      "fma.rn.f32.f16 %0, c3, x3, %0;\n\tfma.rn.f32.f16 %1, c7, x7, %1;\n\t}"
+  const uint32_t ca = and_or(w, k.mlo, k.f1024);     // (1024 + q0, 1024 + q1)
+  const uint32_t cb = and_or(w, k.mhi, k.f64);       // (64 + q2, 64 + q3)
+  const uint32_t cc = and_or(w8, k.mlo, k.f1024);    // (1024 + q4, 1024 + q5)
+  const uint32_t cd = and_or(w8, k.mhi, k.f64);      // (64 + q6, 64 + q7)
+  asm("{\n\t.reg .b16 c0, c1, c2, c3, c4, c5, c6, c7, x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
+      "mov.b32 {c0, c1}, %2;\n\tmov.b32 {c2, c3}, %3;\n\t"
+      "mov.b32 {c4, c5}, %4;\n\tmov.b32 {c6, c7}, %5;\n\t"
+      "mov.b32 {x0, x1}, %6;\n\tmov.b32 {x2, x3}, %7;\n\t"
+      "mov.b32 {x4, x5}, %8;\n\tmov.b32 {x6, x7}, %9;\n\t"
+      "fma.rn.f32.f16 %0, c0, x0, %0;\n\tfma.rn.f32.f16 %1, c1, x1, %1;\n\t"
+      "fma.rn.f32.f16 %0, c2, x2, %0;\n\tfma.rn.f32.f16 %1, c3, x3, %1;\n\t"
+      "fma.rn.f32.f16 %0, c4, x4, %0;\n\tfma.rn.f32.f16 %1, c5, x5, %1;\n\t"
+      "fma.rn.f32.f16 %0, c6, x6, %0;\n\tfma.rn.f32.f16 %1, c7, x7, %1;\n\t}"
       : "+f"(a0), "+f"(a1)
       : "r"(ca), "r"(cb), "r"(cc), "r"(cd), "r"(xw.x), "r"(xw.y), "r"(xw.z), "r"(xw.w));
 }
 
-// The 8 codes of one word as exact fp32 (q - z) pairs, in input order:
-// f32(128 + q) + cz with cz = -(128 + z), by the mixed-precision add.
+// The 8 codes of one (interleaved) word as exact fp32 (q - z) pairs, in input
+// order: f32(128 + q) + cz with cz = -(128 + z), by the mixed-precision add.
+// nib_pair(w, i) holds the adjacent inputs (2i, 2i+1).
 __device__ __forceinline__ void widen_word(uint32_t w, float cz, float2& d01, float2& d23,
                                            float2& d45, float2& d67, const LopConsts& k) {
   const uint32_t v0 = nib_pair(w, 0, k), v1 = nib_pair(w, 1, k), v2 = nib_pair(w, 2, k),
                  v3 = nib_pair(w, 3, k);
-  asm("{\n\t.reg .b16 q0, q4, q1, q5, q2, q6, q3, q7;\n\t"
-      "mov.b32 {q0, q4}, %8;\n\tmov.b32 {q1, q5}, %9;\n\t"
-      "mov.b32 {q2, q6}, %10;\n\tmov.b32 {q3, q7}, %11;\n\t"
+  asm("{\n\t.reg .b16 q0, q1, q2, q3, q4, q5, q6, q7;\n\t"
+      "mov.b32 {q0, q1}, %8;\n\tmov.b32 {q2, q3}, %9;\n\t"
+      "mov.b32 {q4, q5}, %10;\n\tmov.b32 {q6, q7}, %11;\n\t"
       "add.rn.f32.bf16 %0, q0, %12;\n\tadd.rn.f32.bf16 %1, q1, %12;\n\t"
       "add.rn.f32.bf16 %2, q2, %12;\n\tadd.rn.f32.bf16 %3, q3, %12;\n\t"
       "add.rn.f32.bf16 %4, q4, %12;\n\tadd.rn.f32.bf16 %5, q5, %12;\n\t"
@@ -260,8 +263,8 @@ __device__ __forceinline__ void store_x_slice(const XSlice<MP, MIXED>& xs, uint8
       for (int wd = 0; wd < 2; ++wd) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const __half lo = __float2half_rn(__fmul_rn(xf[8 * wd + i], scale));
-          const __half hi = __float2half_rn(__fmul_rn(xf[8 * wd + i + 4], scale));
+          const __half lo = __float2half_rn(__fmul_rn(xf[8 * wd + 2 * i], scale));
+          const __half hi = __float2half_rn(__fmul_rn(xf[8 * wd + 2 * i + 1], scale));
           hw[4 * wd + i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
           const float f = __half2float(lo) + __half2float(hi);
           if (i & 1) sb += f; else sa += f;

@@ -159,8 +159,20 @@ struct LayoutParams {
   Geom g;
 };
 
+// Nibble interleave of one code word: even nibbles 0,2,4,6 -> slots 0..3, odd
+// nibbles 1,3,5,7 -> slots 4..7.
+__device__ __forceinline__ uint32_t interleave_word(uint32_t w) {
+  uint32_t e = w & 0x0F0F0F0Fu, o = (w >> 4) & 0x0F0F0F0Fu;
+  e = (e | (e >> 4)) & 0x00FF00FFu;
+  e = (e | (e >> 8)) & 0x0000FFFFu;
+  o = (o | (o >> 4)) & 0x00FF00FFu;
+  o = (o | (o >> 8)) & 0x0000FFFFu;
+  return e | (o << 16);
+}
+
 // One CTA per tile (slab s, row tile b): copy the tile's codes row by row in
-// 16-byte chunks, then gather its metadata.  Rows past N are written as 0.
+// 16-byte chunks (nibbles interleaved), then gather its metadata.  Rows past
+// N are written as 0.
 __global__ void __launch_bounds__(256) relayout_kernel(LayoutParams p) {
   const Geom& g = p.g;
   const int s = blockIdx.x / g.NB;
@@ -175,9 +187,12 @@ __global__ void __launch_bounds__(256) relayout_kernel(LayoutParams p) {
     const int cc = c % chunks_per_row;
     const int n = b * kTileRows + r;
     uint4 v = make_uint4(0, 0, 0, 0);
-    if (n < g.N)
+    if (n < g.N) {
       v = __ldg(reinterpret_cast<const uint4*>(p.qweight + (size_t)n * words_per_row +
                                                s * kSlabGroups * 16) + cc);
+      v = make_uint4(interleave_word(v.x), interleave_word(v.y), interleave_word(v.z),
+                     interleave_word(v.w));
+    }
     *reinterpret_cast<uint4*>(tile + r * gs * kCodeBytesPerGroupRow + cc * 16) = v;
   }
   uint8_t* mbase = tile + kTileRows * gs * kCodeBytesPerGroupRow;
