@@ -194,6 +194,31 @@ wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* p
 wq_status wq_last_device_status(wq_stream_t stream);
 
 /*
+ * wq_gemv_w4a16_static -- wq_gemv_w4a16 without a workspace argument, for
+ * callers that cannot allocate device memory (a custom-op hook or plugin whose
+ * host forbids or owns all device allocations, or a captured region with a
+ * fixed memory pool).  The quantization pages have no counterpart: this is a
+ * deployment convenience of this library.
+ *
+ * Same arguments, semantics and result as wq_gemv_w4a16, minus workspace and
+ * ws_bytes.  The split-K scratch lives in one static device array of
+ * WQ_STATIC_SCRATCH_BYTES inside the library (held by every GPU that loads the
+ * library until the process exits); shapes with wq_workspace_bytes(M, N, K)
+ * above that are refused with WQ_ERR_WORKSPACE_TOO_SMALL.  Nothing is
+ * allocated or freed: each call clears the counters it uses with an
+ * asynchronous memset on `stream` and launches the GEMV kernel.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array: calls that may overlap on the GPU (on
+ *     different streams, or from different threads without ordering) race
+ *     and may return wrong results.  Order them on one stream.
+ */
+#define WQ_STATIC_SCRATCH_BYTES (8u << 20)
+wq_status wq_gemv_w4a16_static(const void* x, const float* inv_act_scale, const void* packed,
+                               int M, int N, int K, int group_size, int symmetric, int layout,
+                               float* y, wq_stream_t stream);
+
+/*
  * wq_debug_set_wait_limit_ns -- test hook, not part of the stable ABI: the
  * time a kernel's bounded wait (on its shared-memory pipeline barriers) gives
  * before it records WQ_ERR_TIMEOUT and returns; default 2 s, 0 is treated as

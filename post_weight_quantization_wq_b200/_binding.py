@@ -26,6 +26,7 @@ WQ_ERR_CUDA = 7
 WQ_GROUP_SIZE = 128
 WQ_LAYOUT_TILED = 1
 WQ_WORKSPACE_COUNTER_BYTES = 262144
+WQ_STATIC_SCRATCH_BYTES = 8 << 20
 
 # name -> (restype, argtypes); the exported symbols of include/wq.h
 _P = ctypes.c_void_p
@@ -40,6 +41,7 @@ SIGNATURES = {
     "wq_workspace_bytes": (_S, [_I, _I, _I]),
     "wq_gemv_w4a16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _S, _P]),
     "wq_gemm_w4a16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _S, _P]),
+    "wq_gemv_w4a16_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "wq_last_device_status": (_I, [_P]),
     "wq_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
 }
@@ -132,6 +134,13 @@ def wq_gemm_w4a16(x, inv_act_scale, packed, M, N, K, group_size, symmetric, layo
     return load().wq_gemm_w4a16(_ptr(x), _ptr(inv_act_scale), _ptr(packed), M, N, K,
                                 group_size, int(symmetric), layout, _ptr(y), _ptr(workspace),
                                 ws_bytes, _stream(stream))
+
+
+def wq_gemv_w4a16_static(x, inv_act_scale, packed, M, N, K, group_size, symmetric, layout, y,
+                         stream=None) -> int:
+    return load().wq_gemv_w4a16_static(_ptr(x), _ptr(inv_act_scale), _ptr(packed), M, N, K,
+                                       group_size, int(symmetric), layout, _ptr(y),
+                                       _stream(stream))
 
 
 def wq_last_device_status(stream=None) -> int:

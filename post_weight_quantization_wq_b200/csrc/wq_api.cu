@@ -142,6 +142,20 @@ wq_status check_linear(const void* x, const float* inv_s, const void* packed, in
 
 }  // namespace
 
+namespace wq {
+// Error-word address, SM count and wait limit of the current device (set up
+// on first use), for entry points defined in other files of the library.
+cudaError_t device_info(int** err, int* num_sms, unsigned long long* wait_ns) {
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return e;
+  *err = d->err;
+  *num_sms = d->num_sms;
+  *wait_ns = g_wait_ns.load();
+  return cudaSuccess;
+}
+}  // namespace wq
+
 extern "C" {
 
 const char* wq_status_string(int status) {

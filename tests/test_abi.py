@@ -113,3 +113,15 @@ def test_pack_layout_validation_before_launch():
     assert st == abi.WQ_ERR_INVALID_ARG        # packed buffer too small
     st = abi.wq_pack_layout(0x1000, 0x2000, None, 256, 1024, 128, 0, 1, 0x4000, 1 << 20, 0)
     assert st == abi.WQ_ERR_INVALID_ARG        # asymmetric needs zeros
+
+
+def test_static_gemv_validation_before_launch():
+    """The allocation-free GEMV refuses, before touching the GPU, shapes whose
+    scratch exceeds its static array, and bad arguments."""
+    assert abi.wq_workspace_bytes(8, 8192, 28672) > abi.WQ_STATIC_SCRATCH_BYTES
+    st = abi.wq_gemv_w4a16_static(0x1000, None, 0x2000, 8, 8192, 28672, 128, 0, 1, 0x3000, 0)
+    assert st == abi.WQ_ERR_WORKSPACE_TOO_SMALL
+    st = abi.wq_gemv_w4a16_static(0x1000, None, 0x2000, 9, 8192, 28672, 128, 0, 1, 0x3000, 0)
+    assert st == abi.WQ_ERR_UNSUPPORTED_SHAPE
+    st = abi.wq_gemv_w4a16_static(0x1004, None, 0x2000, 1, 256, 1024, 128, 0, 1, 0x3000, 0)
+    assert st == abi.WQ_ERR_MISALIGNED
