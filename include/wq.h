@@ -140,9 +140,11 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
                          size_t packed_bytes, wq_stream_t stream);
 
 /*
- * wq_workspace_bytes -- workspace needed by wq_gemv_w4a16 / wq_gemm_w4a16
- * for these sizes (split-K partial sums plus completion counters), or 0
- * when the call needs none.  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
+ * wq_workspace_bytes -- workspace needed by wq_gemv_w4a16 (M = 1..8) or
+ * wq_gemm_w4a16 (M = 16..64) for these sizes, or 0 when the call needs none
+ * (and for M outside both ranges).  It holds completion counters and split-K
+ * partial sums; for wq_gemm_w4a16 also the per-group sums of x (so every
+ * GEMM call needs one).  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
  * the counters: they must be zero before the first call that uses a
  * workspace (allocate it zero-filled), and every call that completes leaves
  * them zero again, so one workspace serves any number of later calls of any
@@ -173,10 +175,10 @@ wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* p
 
 /*
  * wq_gemm_w4a16 -- the same linear for M = 16..64 activation rows on the
- * tensor cores (tcgen05): weights are dequantized to bf16 tiles holding the
- * exact integers (q - z), multiplied with x on the tensor cores with fp32
- * accumulation per group, and each group's partial sum is scaled by s16 in
- * fp32.  Arguments as wq_gemv_w4a16; inv_act_scale must be NULL
+ * tensor cores (tcgen05): per group, the weights are dequantized into tensor
+ * memory as bf16 tiles holding the exact integers 128 + q, multiplied with x
+ * on the tensor cores with fp32 accumulation, and the group's exact
+ * contribution s16 * (D - (128 + z) * sum_k x[m][k]) is added in fp32.  Arguments as wq_gemv_w4a16; inv_act_scale must be NULL
  * (WQ_ERR_INVALID_ARG otherwise: the bf16 tensor-core operand cannot hold
  * x * inv_act_scale exactly).
  */

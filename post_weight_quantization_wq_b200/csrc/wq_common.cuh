@@ -100,6 +100,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase has not completed is suspended
+// (it issues nothing) until the phase completes or about `hint_ns`
+// nanoseconds have passed.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity,
+                                                      uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -107,14 +122,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // Wait until the phase with the given parity of `bar` has completed, for at
-// most `limit_ns` nanoseconds.  Returns false on timeout.
+// most `limit_ns` nanoseconds.  Returns false on timeout.  The waiting
+// thread sleeps in the barrier instead of spinning, so waiting warps leave
+// the issue slots to the working ones.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint32_t hint = limit_ns < 20000u ? (uint32_t)limit_ns + 1u : 20000u;
   while (true) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, hint)) return true;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }

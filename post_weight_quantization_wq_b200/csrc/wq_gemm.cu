@@ -17,24 +17,31 @@
 // added in fp32 to each row's running sum; the zero point and the 128 bias
 // never enter the bf16 operands, so any stored z is handled exactly.
 //
-// Warp roles of one CTA (persistent, one per SM, contiguous run of layout
-// tiles u = b * NS + s like the GEMV):
-//   warp 0     producer: 1-D bulk copy of each code tile (codes + metadata)
-//              into a 2-stage ring, and per group two 2-D TMA loads of x
-//              (SWIZZLE_128B, rows >= M zero-filled) into a 4-slot ring;
-//   warp 1     allocates tensor memory; one lane issues 8 tcgen05.mma
-//              (M=128, N=Mpad, K=16) per group into one of two accumulator
-//              buffers and commits them to mbarriers;
-//   warps 2-5  dequantize: 4 LOP3 + 3 shifts turn a code word into four
-//              bf16 pairs (inputs 2t, 2t+1 of the interleaved word) stored
-//              into the K-major SWIZZLE_128B A tile (double-buffered);
-//   warps 6-9  epilogue: one thread per output row reads the group's
-//              accumulator row with tcgen05.ld, folds in s16, z and sum(x),
-//              and keeps the row's running sums; row tiles split between
-//              CTAs are finished through the workspace as in the GEMV.
-// Every wait is bounded; on timeout the kernel records the device error word
-// and winds down (waiting, bounded, for its copies and MMAs in flight).
+// Data flow of one CTA (persistent, one per SM, contiguous run of layout
+// tiles u = b * NS + s like the GEMV), per group of 128 inputs:
+//   codes   2-D TMA load of the group's 128 rows x 64 B of codes out of the
+//           packed tile (SWIZZLE_64B, so that a warp reading 32 rows at one
+//           column offset touches every bank once) into a 12..16-slot ring;
+//   A       the dequantizing warps turn each row's 16 code words into 64
+//           bf16 pairs and store them into tensor memory (tcgen05.st): the
+//           A operand never passes through shared memory;
+//   x       2-D TMA loads of the bf16 activation tile (SWIZZLE_128B, rows >= M
+//           zero-filled) into a 4-slot ring, and a bulk copy of the group's
+//           precomputed sum(x) row into an 8-slot ring;
+//   MMA     one lane issues 8 tcgen05.mma (M=128, N=Mpad, K=16, A in tensor
+//           memory, B in shared memory) into one of 4 accumulators;
+//   fold    one thread per output row reads its accumulator row (tcgen05.ld)
+//           and adds s16 * (D - (128 + z) * sum(x)) to the row's running sums;
+//           row tiles split between CTAs are finished through the workspace
+//           as in the GEMV.
+// Warps: 0 code producer, 1 tensor-memory owner and MMA issuer, 2
+// activation producer, 4-11 dequantize (inputs 0-63 and 64-127 of each
+// group, one warp per lane quadrant), 12-19 fold (columns 0..Mpad/2-1 and
+// Mpad/2..Mpad-1 of the accumulator, one warp per lane quadrant).  Every wait is bounded; on timeout the kernel records
+// the device error word and winds down (waiting, bounded, for its copies and
+// MMAs in flight).
 #include <cuda.h>
+#include <cstring>
 #include <cudaTypedefs.h>
 
 #include "wq_common.cuh"
@@ -43,42 +50,54 @@ namespace wq {
 
 struct GemmParams {
   const uint8_t* packed;
+  const float* xsum;       // fp32 [NG][64]: sum of x over each group, per row of x
   float* y;
   float* partials;         // fp32 [NS][64][Npad]
   unsigned* counters;
   int* err;
   Geom g;
   int M;
+  int ns_full;             // slabs with kSlabGroups groups
+  int tile_rows;           // 256-byte (full slab) or gs*64-byte rows per tile
   long long tiles;
   unsigned long long wait_ns;
   unsigned long long drain_ns;
   uint32_t lop_mask_lo, lop_bf16_128;
 };
 
-constexpr int kGemmWarps = 10;
+constexpr int kGemmWarps = 20;
 constexpr int kGemmThreads = kGemmWarps * 32;
-constexpr int kCodeStages = 2;
-constexpr int kBSlots = 4;
+constexpr int kDqWarps = 8;
+constexpr int kEpiWarps = 8;
+constexpr int kABufs = 4;                   // A operands in tensor memory
+constexpr int kAccBufs = 4;                 // accumulators in tensor memory
+constexpr int kBSlots = 4;                  // bf16 x tiles
+constexpr int kXsSlots = 8;                 // sum(x) rows
+constexpr int kMetaSlots = 8;               // per-tile scales (and zeros)
+constexpr int kMetaSlotBytes = kTileRows * kSlabGroups * 4;   // 2 KB
 constexpr int kGemmPartialM = 64;           // workspace row stride (max M)
+constexpr int kCodeGroupBytes = kTileRows * kCodeBytesPerGroupRow;   // 8 KB
+constexpr uint32_t kTmemCols = 512;
 
 template <int MPAD>
 struct GemmSmem {
-  static constexpr int kA = kTileRows * kGroup * 2;          // 32 KB bf16 A tile
-  static constexpr int kB = MPAD * kGroup * 2;               // bf16 B tile
-  static constexpr int kAOff = 0;
-  static constexpr int kBOff = kAOff + 2 * kA;
-  static constexpr int kTileOff = kBOff + kBSlots * kB;
-  static constexpr int kTileBytes = kTileRows * kSlabGroups * (kCodeBytesPerGroupRow + 4);
-  // fp32 scratch for sum(x): totals [2][MPAD], partial sums [2][8][MPAD]
-  static constexpr int kXsumOff = kTileOff + kCodeStages * kTileBytes;
-  static constexpr int kXsumBytes = (2 * MPAD + 2 * 8 * MPAD) * 4;
-  static constexpr int kBarOff = (kXsumOff + kXsumBytes + 15) / 16 * 16;
-  static constexpr int kNumBars = 2 * kCodeStages + 2 * 2 + 2 * kBSlots + 2 * 2 + 2;
-  // accumulator buffers in tensor memory: column stride and allocation
-  static constexpr int kAccStride = MPAD <= 32 ? MPAD : 64;
-  static constexpr uint32_t kTmemCols = 2 * kAccStride <= 32 ? 32 : 2 * kAccStride <= 64 ? 64 : 128;
+  static constexpr int kCodeSlots = MPAD <= 32 ? 16 : 12;
+  static constexpr int kB = MPAD * kGroup * 2;                // bf16 x tile
+  static constexpr int kBOff = 0;
+  static constexpr int kCodeOff = kBOff + kBSlots * kB;
+  static constexpr int kXsOff = kCodeOff + kCodeSlots * kCodeGroupBytes;
+  static constexpr int kXs = kGemmPartialM * 4;                // one sum(x) row
+  static constexpr int kMetaOff = kXsOff + kXsSlots * kXs;
+  static constexpr int kBarOff = kMetaOff + kMetaSlots * kMetaSlotBytes;
+  static constexpr int kNumBars = 2 * kCodeSlots + 2 * kABufs + 2 * kBSlots + 2 * kXsSlots +
+                                  2 * kAccBufs + 2 * kMetaSlots;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                // slack for 1024-B alignment
+  // tensor memory columns: A buffers (64 columns = 128 bf16 each), then
+  // the accumulators
+  static constexpr int kAccStride = MPAD <= 32 ? 32 : 64;
+  static constexpr int kAccCol = kABufs * 64;
+  static_assert(kAccCol + kAccBufs * kAccStride <= (int)kTmemCols, "tensor memory");
 };
 
 // UMMA shared-memory descriptor: K-major, SWIZZLE_128B, 8-row atoms of
@@ -96,12 +115,14 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16() {
          ((uint32_t)(128 >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
+// D (tensor memory) (+)= A (tensor memory, 128 rows x 16 bf16, two per
+// column) * B (shared memory descriptor)^T
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -118,22 +139,36 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 16 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
+// 8 consecutive fp32 columns of this thread's TMEM lane (asynchronous: the
+// registers are valid after tmem_wait_ld).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15}, [%16];"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
+        "=r"(r[7])
       : "r"(taddr));
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
@@ -155,56 +190,87 @@ __device__ __forceinline__ int owner_of(long long u, long long T, int G) {
   return (int)(((u + 1) * G + T - 1) / T) - 1;
 }
 
+// Walks the groups of this CTA's run of tiles in order: group j is group gg
+// of slab s of row tile b.
+struct GroupCursor {
+  int b, s, gg, gs;
+  __device__ void init(const Geom& g, long long t0) {
+    b = (int)(t0 / g.NS);
+    s = (int)(t0 % g.NS);
+    gg = 0;
+    gs = slab_groups(g, s);
+  }
+  // returns true when the step crossed into the next tile
+  __device__ bool next(const Geom& g) {
+    if (++gg < gs) return false;
+    gg = 0;
+    if (++s == g.NS) { s = 0; ++b; }
+    gs = slab_groups(g, s);
+    return true;
+  }
+};
+
 template <int MPAD>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_w4a16_tc_kernel(const GemmParams prm, const __grid_constant__ CUtensorMap xmap) {
+    gemm_w4a16_tc_kernel(const GemmParams prm, const __grid_constant__ CUtensorMap xmap,
+                         const __grid_constant__ CUtensorMap cmap_full,
+                         const __grid_constant__ CUtensorMap cmap_tail) {
   using SM = GemmSmem<MPAD>;
+  constexpr int NC = SM::kCodeSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const Geom g = prm.g;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
-  uint64_t* tfull = bars;                       // [2] code tile landed
-  uint64_t* tempty = tfull + kCodeStages;       // [2] code tile consumed (4 dequant warps)
-  uint64_t* afull = tempty + kCodeStages;       // [2] A tile written (4 dequant warps)
-  uint64_t* aempty = afull + 2;                 // [2] A tile read by the MMAs (commit)
-  uint64_t* bfull = aempty + 2;                 // [4] x tile landed (TMA)
-  uint64_t* bempty = bfull + kBSlots;           // [4] x tile used by MMA (commit) + epilogue
-  uint64_t* accfull = bempty + kBSlots;         // [2] accumulator ready (commit)
-  uint64_t* accempty = accfull + 2;             // [2] accumulator read (4 epilogue warps)
-  uint64_t* xp_bar = accempty + 2;              // partial sums of x written (4 epilogue warps)
-  uint64_t* xs_bar = xp_bar + 1;                // totals of x written (warps holding et < MPAD)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xs_bar + 1);
+  uint64_t* cfull = bars;                       // [NC] codes of a group landed (TMA)
+  uint64_t* cempty = cfull + NC;                // [NC] codes read (8 dequant warps)
+  uint64_t* afull = cempty + NC;                // [4] A operand stored (8 dequant warps)
+  uint64_t* aempty = afull + kABufs;            // [4] A operand read by the MMAs (commit)
+  uint64_t* bfull = aempty + kABufs;            // [4] x tile landed (TMA)
+  uint64_t* bempty = bfull + kBSlots;           // [4] x tile read by the MMAs (commit)
+  uint64_t* xsfull = bempty + kBSlots;          // [8] sum(x) row landed
+  uint64_t* xsempty = xsfull + kXsSlots;        // [8] sum(x) row read (8 fold warps)
+  uint64_t* accfull = xsempty + kXsSlots;       // [4] accumulator ready (commit)
+  uint64_t* accempty = accfull + kAccBufs;      // [4] accumulator read (8 fold warps)
+  uint64_t* mfull = accempty + kAccBufs;        // [8] metadata of a tile landed
+  uint64_t* mempty = mfull + kMetaSlots;        // [8] metadata read (8 fold warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mempty + kMetaSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xsum = reinterpret_cast<float*>(smem + SM::kXsumOff);       // [2][MPAD]
-  float* xpart = xsum + 2 * MPAD;                                    // [2][8][MPAD]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = gridDim.x;
   const long long t0 = (long long)blockIdx.x * prm.tiles / G;
   const long long t1 = (long long)(blockIdx.x + 1) * prm.tiles / G;
-  const int ntiles = (int)(t1 - t0);
-  constexpr uint32_t kTmemCols = SM::kTmemCols;
-  constexpr int kXsWarps = (MPAD + 31) / 32;    // epilogue warps that total sum(x)
+  // groups of this CTA's run of tiles
+  int ngroups = 0;
+  for (long long u = t0; u < t1; ++u) ngroups += slab_groups(g, (int)(u % g.NS));
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kCodeStages; ++i) {
-      mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+    for (int i = 0; i < NC; ++i) {
+      mbar_init(&cfull[i], 1);
+      mbar_init(&cempty[i], kDqWarps);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&afull[i], 4);
+    for (int i = 0; i < kABufs; ++i) {
+      mbar_init(&afull[i], kDqWarps);
       mbar_init(&aempty[i], 1);
-      mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 4);
     }
     for (int i = 0; i < kBSlots; ++i) {
       mbar_init(&bfull[i], 1);
-      mbar_init(&bempty[i], 2);
+      mbar_init(&bempty[i], 1);
     }
-    mbar_init(xp_bar, 4);
-    mbar_init(xs_bar, kXsWarps);
+    for (int i = 0; i < kXsSlots; ++i) {
+      mbar_init(&xsfull[i], 1);
+      mbar_init(&xsempty[i], kEpiWarps);
+    }
+    for (int i = 0; i < kAccBufs; ++i) {
+      mbar_init(&accfull[i], 1);
+      mbar_init(&accempty[i], kEpiWarps);
+    }
+    for (int i = 0; i < kMetaSlots; ++i) {
+      mbar_init(&mfull[i], 1);
+      mbar_init(&mempty[i], kEpiWarps);
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -226,251 +292,272 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ code producer
     if (lane == 0) {
-      int b = (int)(t0 / g.NS), s = (int)(t0 % g.NS);
-      int j = 0, issued_t = 0, issued_b = 0;
+      GroupCursor c;
+      c.init(g, t0);
+      int issued = 0, tile = 0, issued_m = 0;
       bool ok = true;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int st = i % kCodeStages;
-        if (i >= kCodeStages)
-          ok = mbar_wait_bounded(&tempty[st], ((i / kCodeStages) - 1) & 1, prm.wait_ns);
-        if (!ok || *abort_flag) { ok = false; break; }
-        const int gs = slab_groups(g, s);
-        const uint32_t tbytes = (uint32_t)tile_bytes(g, gs);
-        mbar_arrive_expect_tx(&tfull[st], tbytes);
-        bulk_copy_g2s(smem + SM::kTileOff + st * SM::kTileBytes,
-                      prm.packed + tile_offset(g, s, b), tbytes, &tfull[st]);
-        issued_t = i + 1;
-        for (int gg = 0; gg < gs; ++gg, ++j) {
-          const int bs = j % kBSlots;
-          if (j >= kBSlots)
-            ok = mbar_wait_bounded(&bempty[bs], ((j / kBSlots) - 1) & 1, prm.wait_ns);
+      for (int j = 0; j < ngroups; ++j, c.next(g)) {
+        if (c.gg == 0) {
+          // the tile's metadata block (128 rows x gs groups) into a meta slot
+          const int ms = tile % kMetaSlots;
+          if (tile >= kMetaSlots)
+            ok = mbar_wait_bounded(&mempty[ms], ((tile / kMetaSlots) - 1) & 1, prm.wait_ns);
           if (!ok || *abort_flag) { ok = false; break; }
-          uint8_t* bdst = smem + SM::kBOff + bs * SM::kB;
-          mbar_arrive_expect_tx(&bfull[bs], 2 * MPAD * 128);
-          const int k0 = s * kSlabK + gg * kGroup;
-          tma_load_2d(bdst, &xmap, k0, 0, &bfull[bs]);
-          tma_load_2d(bdst + MPAD * 128, &xmap, k0 + 64, 0, &bfull[bs]);
-          issued_b = j + 1;
+          const uint32_t mbytes = (uint32_t)(kTileRows * c.gs * g.meta);
+          mbar_arrive_expect_tx(&mfull[ms], mbytes);
+          bulk_copy_g2s(smem + SM::kMetaOff + ms * kMetaSlotBytes,
+                        prm.packed + tile_offset(g, c.s, c.b) +
+                            (long long)kTileRows * c.gs * kCodeBytesPerGroupRow,
+                        mbytes, &mfull[ms]);
+          issued_m = ++tile;
         }
-        if (++s == g.NS) { s = 0; ++b; }
+        const int cs = j % NC;
+        if (j >= NC) ok = mbar_wait_bounded(&cempty[cs], ((j / NC) - 1) & 1, prm.wait_ns);
+        if (!ok || *abort_flag) { ok = false; break; }
+        mbar_arrive_expect_tx(&cfull[cs], kCodeGroupBytes);
+        uint8_t* dst = smem + SM::kCodeOff + cs * kCodeGroupBytes;
+        if (c.s < prm.ns_full)
+          tma_load_2d(dst, &cmap_full, c.gg * kCodeBytesPerGroupRow,
+                      (c.s * g.NB + c.b) * prm.tile_rows, &cfull[cs]);
+        else
+          tma_load_2d(dst, &cmap_tail, c.gg * kCodeBytesPerGroupRow, c.b * prm.tile_rows,
+                      &cfull[cs]);
+        issued = j + 1;
       }
       if (!ok) {
         fail();
-        for (int st = 0; st < kCodeStages && st < issued_t; ++st)
-          mbar_wait_bounded(&tfull[st], ((issued_t - 1 - st) / kCodeStages) & 1, prm.drain_ns);
-        for (int bs = 0; bs < kBSlots && bs < issued_b; ++bs)
-          mbar_wait_bounded(&bfull[bs], ((issued_b - 1 - bs) / kBSlots) & 1, prm.drain_ns);
+        for (int k = issued - NC < 0 ? 0 : issued - NC; k < issued; ++k)
+          mbar_wait_bounded(&cfull[k % NC], (k / NC) & 1, prm.drain_ns);
+        for (int k = issued_m - kMetaSlots < 0 ? 0 : issued_m - kMetaSlots; k < issued_m; ++k)
+          mbar_wait_bounded(&mfull[k % kMetaSlots], (k / kMetaSlots) & 1, prm.drain_ns);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      GroupCursor c;
+      c.init(g, t0);
+      int issued_b = 0, issued_x = 0;
+      bool ok = true;
+      for (int j = 0; j < ngroups; ++j, c.next(g)) {
+        const int bs = j % kBSlots, xs = j % kXsSlots;
+        const int k0 = c.s * kSlabK + c.gg * kGroup;
+        if (j >= kBSlots) ok = mbar_wait_bounded(&bempty[bs], ((j / kBSlots) - 1) & 1, prm.wait_ns);
+        if (!ok || *abort_flag) { ok = false; break; }
+        uint8_t* bdst = smem + SM::kBOff + bs * SM::kB;
+        mbar_arrive_expect_tx(&bfull[bs], 2 * MPAD * 128);
+        tma_load_2d(bdst, &xmap, k0, 0, &bfull[bs]);
+        tma_load_2d(bdst + MPAD * 128, &xmap, k0 + 64, 0, &bfull[bs]);
+        issued_b = j + 1;
+        if (j >= kXsSlots)
+          ok = mbar_wait_bounded(&xsempty[xs], ((j / kXsSlots) - 1) & 1, prm.wait_ns);
+        if (!ok || *abort_flag) { ok = false; break; }
+        mbar_arrive_expect_tx(&xsfull[xs], MPAD * 4);
+        bulk_copy_g2s(smem + SM::kXsOff + xs * SM::kXs,
+                      prm.xsum + (size_t)(c.s * kSlabGroups + c.gg) * kGemmPartialM, MPAD * 4,
+                      &xsfull[xs]);
+        issued_x = j + 1;
+      }
+      if (!ok) {
+        fail();
+        for (int k = issued_b - kBSlots < 0 ? 0 : issued_b - kBSlots; k < issued_b; ++k)
+          mbar_wait_bounded(&bfull[k % kBSlots], (k / kBSlots) & 1, prm.drain_ns);
+        for (int k = issued_x - kXsSlots < 0 ? 0 : issued_x - kXsSlots; k < issued_x; ++k)
+          mbar_wait_bounded(&xsfull[k % kXsSlots], (k / kXsSlots) & 1, prm.drain_ns);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int s = (int)(t0 % g.NS);
       int j = 0;
       bool ok = true;
       constexpr uint32_t idesc = umma_idesc_bf16<MPAD>();
-      const uint32_t a0 = smem_u32(smem + SM::kAOff), b0 = smem_u32(smem + SM::kBOff);
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int gs = slab_groups(g, s);
-        for (int gg = 0; gg < gs; ++gg, ++j) {
-          const int ab = j & 1, bs = j % kBSlots, acc = j & 1;
-          ok = mbar_wait_bounded(&afull[ab], (j >> 1) & 1, prm.wait_ns) &&
-               mbar_wait_bounded(&bfull[bs], (j / kBSlots) & 1, prm.wait_ns) &&
-               (j < 2 || mbar_wait_bounded(&accempty[acc], ((j >> 1) - 1) & 1, prm.wait_ns));
-          if (!ok || *abort_flag) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t abase = a0 + ab * SM::kA, bbase = b0 + bs * SM::kB;
+      const uint32_t b0 = smem_u32(smem + SM::kBOff);
+      for (; j < ngroups; ++j) {
+        const int ab = j % kABufs, bs = j % kBSlots, acc = j % kAccBufs;
+        ok = mbar_wait_bounded(&afull[ab], (j / kABufs) & 1, prm.wait_ns) &&
+             mbar_wait_bounded(&bfull[bs], (j / kBSlots) & 1, prm.wait_ns) &&
+             (j < kAccBufs ||
+              mbar_wait_bounded(&accempty[acc], ((j / kAccBufs) - 1) & 1, prm.wait_ns));
+        if (!ok || *abort_flag) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t bbase = b0 + bs * SM::kB;
+        const uint32_t ta = tmem_base + ab * 64;
+        const uint32_t td = tmem_base + SM::kAccCol + acc * SM::kAccStride;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // K = 16 slice kk: 64-input block kk / 4, 32-byte step inside its swizzled rows
-            const uint32_t koff = (kk & 3) * 32;
-            const uint64_t ad = umma_desc_sw128(abase + (kk >> 2) * (kTileRows * 128) + koff);
-            const uint64_t bd = umma_desc_sw128(bbase + (kk >> 2) * (MPAD * 128) + koff);
-            umma_bf16(tmem_base + acc * SM::kAccStride, ad, bd, idesc, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&aempty[ab]);
-          umma_commit(&bempty[bs]);
-          umma_commit(&accfull[acc]);
+        for (int kk = 0; kk < 8; ++kk) {
+          // K = 16 slice kk: 8 columns of A; in B, 64-input block kk / 4 and
+          // a 32-byte step inside its swizzled rows
+          const uint64_t bd = umma_desc_sw128(bbase + (kk >> 2) * (MPAD * 128) + (kk & 3) * 32);
+          umma_bf16_ts(td, ta + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
         }
-        if (++s == g.NS) s = 0;
+        umma_commit(&aempty[ab]);
+        umma_commit(&bempty[bs]);
+        umma_commit(&accfull[acc]);
       }
       if (!ok) {
         fail();
-        // let the MMAs already issued finish before the accumulator is freed
-        if (j > 0) mbar_wait_bounded(&accfull[(j - 1) & 1], ((j - 1) >> 1) & 1, prm.drain_ns);
+        // let the MMAs already issued finish before tensor memory is freed
+        if (j > 0)
+          mbar_wait_bounded(&accfull[(j - 1) % kAccBufs], ((j - 1) / kAccBufs) & 1, prm.drain_ns);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp >= 4 && warp < 4 + kDqWarps) {
     // ------------------------------------------------------------ dequantize
-    const int dt = threadIdx.x - 64;          // 0..127
+    const int quad = warp & 3;                // TMEM lane quadrant of this warp
+    const int h = (warp - 4) >> 2;            // inputs 64h .. 64h+63 of each group
+    const int r = quad * 32 + lane;           // row of the tile (= TMEM lane)
     const uint32_t mlo = prm.lop_mask_lo, b128 = prm.lop_bf16_128;
-    int s = (int)(t0 % g.NS);
-    int j = 0;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quad * 32) << 16) + h * 32;
+    // byte offsets of this row's two 16-byte chunks 2h, 2h+1 in a code slot
+    // (64-byte swizzle: chunk index ^= address bits 7..8)
+    const int sw = (r >> 1) & 3;
+    const int off0 = r * 64 + (((2 * h) ^ sw) << 4);
+    const int off1 = r * 64 + (((2 * h + 1) ^ sw) << 4);
     bool ok = true;
-    for (int i = 0; i < ntiles && ok; ++i) {
-      const int st = i % kCodeStages;
-      const int gs = slab_groups(g, s);
-      bool w_ok = mbar_wait_bounded(&tfull[st], (i / kCodeStages) & 1, prm.wait_ns);
+    for (int j = 0; j < ngroups; ++j) {
+      const int cs = j % NC, ab = j % kABufs;
+      bool w_ok = mbar_wait_bounded(&cfull[cs], (j / NC) & 1, prm.wait_ns);
+      if (w_ok && j >= kABufs)
+        w_ok = mbar_wait_bounded(&aempty[ab], ((j / kABufs) - 1) & 1, prm.wait_ns);
       if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
-      const uint8_t* tile = smem + SM::kTileOff + st * SM::kTileBytes;
-      for (int gg = 0; gg < gs; ++gg, ++j) {
-        const int ab = j & 1;
-        if (j >= 2) w_ok = mbar_wait_bounded(&aempty[ab], ((j >> 1) - 1) & 1, prm.wait_ns);
-        if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
-        uint8_t* A = smem + SM::kAOff + ab * SM::kA;
+      tc_fence_after();
+      const uint8_t* slot = smem + SM::kCodeOff + cs * kCodeGroupBytes;
+      const uint4 c0 = *reinterpret_cast<const uint4*>(slot + off0);
+      const uint4 c1 = *reinterpret_cast<const uint4*>(slot + off1);
+      const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int item = it * 128 + dt;     // (row, 16-byte chunk of the group's 64 B)
-          const int r = item >> 2, c = item & 3;
-          const uint4 cw = *reinterpret_cast<const uint4*>(
-              tile + r * gs * kCodeBytesPerGroupRow + gg * kCodeBytesPerGroupRow + c * 16);
-          const uint32_t wds[4] = {cw.x, cw.y, cw.z, cw.w};
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            // word q of chunk c covers inputs 32c + 8q .. +8 of the group
-            const uint32_t w = wds[q];
-            uint4 v;
-            v.x = and_or3(w, mlo, b128);          // inputs 0, 1 -> 128 + q
-            v.y = and_or3(w >> 4, mlo, b128);     // inputs 2, 3
-            v.z = and_or3(w >> 8, mlo, b128);     // inputs 4, 5
-            v.w = and_or3(w >> 12, mlo, b128);    // inputs 6, 7
-            const int kc = 4 * c + q;             // 8-input chunk 0..15 of the group
-            const int kb = kc >> 3, cc = kc & 7;
-            *reinterpret_cast<uint4*>(A + kb * (kTileRows * 128) + r * 128 +
-                                      ((cc ^ (r & 7)) << 4)) = v;
-          }
+        for (int q = 0; q < 4; ++q) {
+          // word covers 8 inputs; slot t of the interleaved word holds input
+          // 2t (t < 4) or 2(t-4)+1, so each LOP3 yields one bf16 pair
+          // (128 + q_even, 128 + q_odd)
+          const uint32_t w = wds[4 * half + q];
+          v[4 * q + 0] = and_or3(w, mlo, b128);
+          v[4 * q + 1] = and_or3(w >> 4, mlo, b128);
+          v[4 * q + 2] = and_or3(w >> 8, mlo, b128);
+          v[4 * q + 3] = and_or3(w >> 12, mlo, b128);
         }
-        fence_proxy_async_shared();               // make the tile visible to the tensor core
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[ab]);
+        tmem_st16(lane_base + ab * 64 + half * 16, v);
       }
-      if (!ok) break;
+      __syncwarp();                           // every lane's codes are in registers
+      if (lane == 0) mbar_arrive(&cempty[cs]);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[st]);
-      if (++s == g.NS) s = 0;
+      if (lane == 0) mbar_arrive(&afull[ab]);
     }
     if (!ok && lane == 0) fail();
-  } else {
-    // ------------------------------------------------------------ epilogue
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ fold
+    constexpr int EC = MPAD / 2;              // accumulator columns of this thread
     const int q4 = warp & 3;                  // TMEM lane quadrant of this warp
-    const int et = (warp - 6) * 32 + lane;    // 0..127 among the epilogue threads
+    const int half = (warp - 12) >> 2;        // columns half*EC .. half*EC+EC-1
+    const int m0 = half * EC;
     const int row = q4 * 32 + lane;           // row of the tile (= TMEM lane)
-    constexpr int kParts = 128 / MPAD;        // xsum partial sums per activation row
-    constexpr int kPartK = kGroup / kParts;
-    float run[MPAD];
+    float run[EC];
 #pragma unroll
-    for (int m = 0; m < MPAD; ++m) run[m] = 0.0f;
-    int b = (int)(t0 / g.NS), s = (int)(t0 % g.NS);
+    for (int m = 0; m < EC; ++m) run[m] = 0.0f;
+    GroupCursor c;
+    c.init(g, t0);
     int piece_s0 = -1;
-    int j = 0;
     bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
-      const int gs = slab_groups(g, s);
-      if (piece_s0 < 0) piece_s0 = s;
-      const uint8_t* meta_g = prm.packed + tile_offset(g, s, b) +
-                              (long long)kTileRows * gs * kCodeBytesPerGroupRow;
-      for (int gg = 0; gg < gs && ok; ++gg, ++j) {
-        const int bs = j % kBSlots, acc = j & 1;
-        // this row's scale and zero for the group (L2-resident: the bulk copy
-        // of the tile has just read them)
-        float sc, cz;
-        if (g.sym) {
-          sc = __half2float(__ldg(reinterpret_cast<const __half*>(meta_g) + row * gs + gg));
-          cz = 136.0f;                         // 128 + 8
-        } else {
-          const __half2 sz = __ldg(reinterpret_cast<const __half2*>(meta_g) + row * gs + gg);
-          sc = __low2float(sz);
-          cz = 128.0f + __high2float(sz);
-        }
-        // sum_k x[m][k] over the group, from the swizzled B tile
-        bool w_ok = mbar_wait_bounded(&bfull[bs], (j / kBSlots) & 1, prm.wait_ns);
-        if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
-        const uint8_t* B = smem + SM::kBOff + bs * SM::kB;
-        float* xp = xpart + (j & 1) * 8 * MPAD;
-        float* xt = xsum + (j & 1) * MPAD;
-        if (et < kParts * MPAD) {
-          const int m = et % MPAD, part = et / MPAD;
-          float sum = 0.0f;
+    float scs[kSlabGroups], czs[kSlabGroups];   // this row's (scale, 128 + zero) per group
+    int tile = 0;
+    for (int j = 0; j < ngroups; ++j) {
+      const int xs = j % kXsSlots, acc = j % kAccBufs;
+      if (piece_s0 < 0) piece_s0 = c.s;
+      if (c.gg == 0) {
+        // the tile's scales (and zeros) for this row, then release the slot
+        const int ms = tile % kMetaSlots;
+        const bool m_ok = mbar_wait_bounded(&mfull[ms], (tile / kMetaSlots) & 1, prm.wait_ns);
+        if (!__all_sync(0xFFFFFFFFu, m_ok) || *abort_flag) { ok = false; break; }
+        const uint8_t* mb = smem + SM::kMetaOff + ms * kMetaSlotBytes;
 #pragma unroll
-          for (int kc = 0; kc < kPartK / 8; ++kc) {
-            const int k = part * kPartK + kc * 8;
-            const int kb = k >> 6, cc = (k & 63) >> 3;
-            const uint4 v = *reinterpret_cast<const uint4*>(B + kb * (MPAD * 128) + m * 128 +
-                                                            ((cc ^ (m & 7)) << 4));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-              sum += __uint_as_float(w4[h] << 16) + __uint_as_float(w4[h] & 0xFFFF0000u);
+        for (int q = 0; q < kSlabGroups; ++q) {
+          if (q < c.gs) {
+            if (g.sym) {
+              scs[q] = __half2float(reinterpret_cast<const __half*>(mb)[row * c.gs + q]);
+              czs[q] = 136.0f;                 // 128 + 8
+            } else {
+              const __half2 sz = reinterpret_cast<const __half2*>(mb)[row * c.gs + q];
+              scs[q] = __low2float(sz);
+              czs[q] = 128.0f + __high2float(sz);
+            }
           }
-          xp[part * MPAD + m] = sum;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(xp_bar);
-        w_ok = mbar_wait_bounded(xp_bar, j & 1, prm.wait_ns);
-        if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
-        if (et == 0) mbar_arrive(&bempty[bs]);       // B no longer needed here
-        if (warp - 6 < kXsWarps) {
-          if (et < MPAD) {
-            float tot = 0.0f;
-#pragma unroll
-            for (int pp = 0; pp < kParts; ++pp) tot += xp[pp * MPAD + et];
-            xt[et] = tot;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xs_bar);
-        }
-        w_ok = mbar_wait_bounded(xs_bar, j & 1, prm.wait_ns);
-        if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
-        // the group's accumulator row
-        w_ok = mbar_wait_bounded(&accfull[acc], (j >> 1) & 1, prm.wait_ns);
-        if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
-        tc_fence_after();
-        // 16 columns at a time: load, wait, fold (keeps few registers live)
-#pragma unroll
-        for (int c = 0; c < MPAD / 16; ++c) {
-          float d[16];
-          tmem_ld16(tmem_base + ((uint32_t)(q4 * 32) << 16) + acc * SM::kAccStride + c * 16, d);
-          tmem_wait_ld();
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-            run[16 * c + m] = fmaf(sc, fmaf(-cz, xt[16 * c + m], d[m]), run[16 * c + m]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&accempty[acc]);
+        if (lane == 0) mbar_arrive(&mempty[ms]);
+        ++tile;
       }
-      if (!ok) break;
-      // ---- end of this CTA's piece of row tile b: write y or a partial
-      const bool piece_end = (s == g.NS - 1) || (i == ntiles - 1);
+      float sc = scs[0], cz = czs[0];
+#pragma unroll
+      for (int q = 1; q < kSlabGroups; ++q)
+        if (c.gg == q) { sc = scs[q]; cz = czs[q]; }
+      GroupCursor nc = c;
+      const bool tile_end = nc.next(g);
+      bool w_ok = mbar_wait_bounded(&xsfull[xs], (j / kXsSlots) & 1, prm.wait_ns) &&
+                  mbar_wait_bounded(&accfull[acc], (j / kAccBufs) & 1, prm.wait_ns);
+      if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
+      tc_fence_after();
+      const float* xt = reinterpret_cast<const float*>(smem + SM::kXsOff + xs * SM::kXs) + m0;
+      const uint32_t tacc = tmem_base + ((uint32_t)(q4 * 32) << 16) + SM::kAccCol +
+                            acc * SM::kAccStride + m0;
+      // batches of up to 16 columns: load, wait, fold (bounds live registers)
+#pragma unroll
+      for (int b0 = 0; b0 < EC; b0 += 16) {
+        constexpr int kMaxB = EC < 16 ? EC : 16;
+        float d[kMaxB];
+#pragma unroll
+        for (int cc = 0; cc < kMaxB / 8; ++cc)
+          if (b0 + cc * 8 < EC) tmem_ld8(tacc + b0 + cc * 8, d + cc * 8);
+        tmem_wait_ld();
+#pragma unroll
+        for (int m = 0; m < kMaxB; ++m)
+          if (b0 + m < EC)
+            run[b0 + m] = fmaf(sc, fmaf(-cz, xt[b0 + m], d[m]), run[b0 + m]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[acc]);
+      if (lane == 0) mbar_arrive(&xsempty[xs]);
+      if (!tile_end) { c = nc; continue; }
+      // ---- last group of a tile: end of this CTA's piece of row tile b?
+      const bool piece_end = (c.s == g.NS - 1) || (j == ngroups - 1);
       if (piece_end) {
-        const bool whole = (piece_s0 == 0) && (s == g.NS - 1);
+        const int b = c.b;
+        const bool whole = (piece_s0 == 0) && (c.s == g.NS - 1);
         const int n = b * kTileRows + row;
         if (whole) {
           if (n < g.N) {
 #pragma unroll
-            for (int m = 0; m < MPAD; ++m)
-              if (m < prm.M) prm.y[(size_t)m * g.N + n] = run[m];
+            for (int m = 0; m < EC; ++m)
+              if (m0 + m < prm.M) prm.y[(size_t)(m0 + m) * g.N + n] = run[m];
           }
         } else {
 #pragma unroll
-          for (int m = 0; m < MPAD; ++m)
-            if (m < prm.M)
-              prm.partials[((size_t)piece_s0 * kGemmPartialM + m) * g.Npad + n] = run[m];
+          for (int m = 0; m < EC; ++m)
+            if (m0 + m < prm.M)
+              prm.partials[((size_t)piece_s0 * kGemmPartialM + m0 + m) * g.Npad + n] = run[m];
           __threadfence();
           __syncwarp();
           const long long ub = (long long)b * g.NS;
           const int c_first = owner_of(ub, prm.tiles, G);
           const int c_last = owner_of(ub + g.NS - 1, prm.tiles, G);
           unsigned prev = 0;
-          unsigned* ctr = prm.counters + (size_t)b * (kTileRows / kRowsPerCounter) + q4;
+          unsigned* ctr =
+              prm.counters + (size_t)b * (kTileRows / kRowsPerCounter) + q4 + 4 * half;
           if (lane == 0) prev = atomicAdd(ctr, 1u);
           prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
           if (prev == (unsigned)(c_last - c_first)) {
             __threadfence();
+            const int m_end = prm.M < m0 + EC ? prm.M : m0 + EC;
             if (n < g.N)
-              for (int m = 0; m < prm.M; ++m) {
+              for (int m = m0; m < m_end; ++m) {
                 float tot = 0.0f;
                 for (int c2 = c_first; c2 <= c_last; ++c2) {
                   const long long tc = (long long)c2 * prm.tiles / G;
@@ -483,10 +570,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
 #pragma unroll
-        for (int m = 0; m < MPAD; ++m) run[m] = 0.0f;
+        for (int m = 0; m < EC; ++m) run[m] = 0.0f;
         piece_s0 = -1;
       }
-      if (++s == g.NS) { s = 0; ++b; }
+      c = nc;
     }
     if (!ok && lane == 0) fail();
   }
@@ -502,13 +589,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// sum_{k in g} x[m][k] for every group g and row m of x, in fp32 (fixed
+// order); rows m >= M are 0.  One warp per group, lane = row of x.
+__global__ void __launch_bounds__(256) gemm_xsum_kernel(const uint16_t* __restrict__ x, int M,
+                                                        int K, float* __restrict__ xsum) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int NG = K / kGroup;
+  if (warp >= NG) return;
+  for (int m = lane; m < kGemmPartialM; m += 32) {
+    float acc = 0.0f;
+    if (m < M) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)m * K + warp * kGroup);
+#pragma unroll 4
+      for (int c = 0; c < kGroup / 8; ++c) {
+        const uint4 v = __ldg(src + c);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          acc += __uint_as_float(w4[h] << 16) + __uint_as_float(w4[h] & 0xFFFF0000u);
+      }
+    }
+    xsum[(size_t)warp * kGemmPartialM + m] = acc;
+  }
+}
+
 // ------------------------------------------------------------------ launcher
+
+static size_t gemm_partials_bytes(const Geom& g) {
+  return g.NS <= 1 ? 0 : (size_t)g.NS * kGemmPartialM * g.Npad * sizeof(float);
+}
 
 size_t gemm_workspace_bytes(int M, int N, int K) {
   (void)M;
   const Geom g = make_geom(N, K, 1);
-  if (g.NS <= 1) return 0;
-  return (size_t)kCounterBytes + (size_t)g.NS * kGemmPartialM * g.Npad * sizeof(float);
+  return (size_t)kCounterBytes + gemm_partials_bytes(g) +
+         (size_t)g.NG * kGemmPartialM * sizeof(float);
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -532,25 +648,57 @@ static cudaError_t launch_gemm_t(const GemmParams& prm, const void* x, int num_s
   using SM = GemmSmem<MPAD>;
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
+  const Geom& g = prm.g;
   // x: bf16 [M][K]; box of 64 inputs x MPAD rows, 128-byte swizzle, rows >= M
   // (and any coordinate past the tensor) read as zero.
-  CUtensorMap map;
-  cuuint64_t dims[2] = {(cuuint64_t)prm.g.K, (cuuint64_t)prm.M};
-  cuuint64_t strides[1] = {(cuuint64_t)prm.g.K * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)MPAD};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  CUtensorMap xmap;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)prm.M};
+    cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)MPAD};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  // Codes: a tile is tile_rows rows of gs * 64 bytes (128 rows of codes,
+  // then the metadata), so the tiles of the full slabs form one 2-D byte
+  // array of 256-byte rows and the tiles of a partial last slab another.
+  // Box: one group (64 bytes) x 128 rows, 64-byte swizzle.
+  CUtensorMap cfull, ctail;
+  memset(&cfull, 0, sizeof(cfull));
+  memset(&ctail, 0, sizeof(ctail));
+  auto encode_codes = [&](CUtensorMap* m, const uint8_t* base, int row_bytes,
+                          long long rows) -> bool {
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)kCodeBytesPerGroupRow, (cuuint32_t)kTileRows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  if (prm.ns_full > 0 &&
+      !encode_codes(&cfull, prm.packed, kSlabGroups * kCodeBytesPerGroupRow,
+                    (long long)prm.ns_full * g.NB * prm.tile_rows))
+    return cudaErrorInvalidValue;
+  if (prm.ns_full < g.NS) {
+    const int gs = slab_groups(g, g.NS - 1);
+    if (!encode_codes(&ctail, prm.packed + tile_offset(g, g.NS - 1, 0),
+                      gs * kCodeBytesPerGroupRow, (long long)g.NB * prm.tile_rows))
+      return cudaErrorInvalidValue;
+  }
   const void* fn = reinterpret_cast<const void*>(&gemm_w4a16_tc_kernel<MPAD>);
   int per_sm = 0;
   cudaError_t e = kernel_setup(fn, SM::kAlloc, kGemmThreads, &per_sm);
   if (e != cudaSuccess) return e;
-  long long grid = (long long)num_sms * per_sm;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  long long grid = (long long)num_sms;        // one CTA per SM (all of tensor memory)
   if (grid > prm.tiles) grid = prm.tiles;
   GemmParams p = prm;
-  void* args[] = {&p, &map};
+  void* args[] = {&p, &xmap, &cfull, &ctail};
   return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(kGemmThreads), args, SM::kAlloc, stream);
 }
 
@@ -562,15 +710,27 @@ cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, 
   prm.packed = static_cast<const uint8_t*>(packed);
   prm.y = y;
   prm.counters = static_cast<unsigned*>(workspace);
-  prm.partials = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes)
-                           : nullptr;
+  prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
+  float* xsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes +
+                                         gemm_partials_bytes(prm.g));
+  prm.xsum = xsum;
   prm.err = err;
   prm.M = M;
   prm.tiles = (long long)prm.g.NS * prm.g.NB;
+  prm.ns_full = prm.g.NG / kSlabGroups;
+  // rows of gs * 64 bytes per tile: 128 of codes + 128 * gs * meta / (gs * 64)
+  prm.tile_rows = kTileRows + kTileRows * prm.g.meta / kCodeBytesPerGroupRow;
   prm.wait_ns = wait_ns;
   prm.drain_ns = 1000000000ull;
   prm.lop_mask_lo = 0x000F000Fu;
   prm.lop_bf16_128 = 0x43004300u;
+  {
+    const int warps = prm.g.NG;
+    gemm_xsum_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(
+        static_cast<const uint16_t*>(x), M, K, xsum);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int mpad = (M + 15) / 16 * 16;
   switch (mpad) {
     case 16: return launch_gemm_t<16>(prm, x, num_sms, stream);

@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
       auto tile_compute = [&](auto ragged_tag) {
       constexpr bool kRagged = decltype(ragged_tag)::value;
       const bool active = !kRagged || p < 2 * gs;
-      float4 xinfo[MIXED ? MP : 1];    // mixed: (bias, sum x, 2^-e, -) of this lane's chunk
+      [[maybe_unused]] float4 xinfo[MIXED ? MP : 1];   // mixed: (bias, sum x, 2^-e, -) of this lane's chunk
       if constexpr (MIXED) {
 #pragma unroll
         for (int m = 0; m < MP; ++m)
