@@ -186,6 +186,20 @@ __device__ __forceinline__ uint32_t and_or3(uint32_t a, uint32_t b, uint32_t c) 
   return d;
 }
 
+// One lane of the (converged) warp returns true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// mbar_wait_bounded by every lane of the warp; true when all saw the phase.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(bar, parity, limit_ns));
+}
+
 __device__ __forceinline__ int owner_of(long long u, long long T, int G) {
   return (int)(((u + 1) * G + T - 1) / T) - 1;
 }
@@ -291,31 +305,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     *abort_flag = 1;
   };
 
+  // The producer and MMA warps run their loops with all 32 lanes (so loop
+  // state stays warp-uniform) and let one elected lane issue each copy or
+  // MMA.
   if (warp == 0) {
     // ------------------------------------------------------------ code producer
-    if (lane == 0) {
-      GroupCursor c;
-      c.init(g, t0);
-      int issued = 0, tile = 0, issued_m = 0;
-      bool ok = true;
-      for (int j = 0; j < ngroups; ++j, c.next(g)) {
-        if (c.gg == 0) {
-          // the tile's metadata block (128 rows x gs groups) into a meta slot
-          const int ms = tile % kMetaSlots;
-          if (tile >= kMetaSlots)
-            ok = mbar_wait_bounded(&mempty[ms], ((tile / kMetaSlots) - 1) & 1, prm.wait_ns);
-          if (!ok || *abort_flag) { ok = false; break; }
+    GroupCursor c;
+    c.init(g, t0);
+    int issued = 0, tile = 0, issued_m = 0;
+    bool ok = true;
+    for (int j = 0; j < ngroups; ++j, c.next(g)) {
+      if (c.gg == 0) {
+        // the tile's metadata block (128 rows x gs groups) into a meta slot
+        const int ms = tile % kMetaSlots;
+        if (tile >= kMetaSlots)
+          ok = warp_wait(&mempty[ms], ((tile / kMetaSlots) - 1) & 1, prm.wait_ns);
+        if (!ok || *abort_flag) { ok = false; break; }
+        if (elect_one()) {
           const uint32_t mbytes = (uint32_t)(kTileRows * c.gs * g.meta);
           mbar_arrive_expect_tx(&mfull[ms], mbytes);
           bulk_copy_g2s(smem + SM::kMetaOff + ms * kMetaSlotBytes,
                         prm.packed + tile_offset(g, c.s, c.b) +
                             (long long)kTileRows * c.gs * kCodeBytesPerGroupRow,
                         mbytes, &mfull[ms]);
-          issued_m = ++tile;
         }
-        const int cs = j % NC;
-        if (j >= NC) ok = mbar_wait_bounded(&cempty[cs], ((j / NC) - 1) & 1, prm.wait_ns);
-        if (!ok || *abort_flag) { ok = false; break; }
+        __syncwarp();
+        issued_m = ++tile;
+      }
+      const int cs = j % NC;
+      if (j >= NC) ok = warp_wait(&cempty[cs], ((j / NC) - 1) & 1, prm.wait_ns);
+      if (!ok || *abort_flag) { ok = false; break; }
+      if (elect_one()) {
         mbar_arrive_expect_tx(&cfull[cs], kCodeGroupBytes);
         uint8_t* dst = smem + SM::kCodeOff + cs * kCodeGroupBytes;
         if (c.s < prm.ns_full)
@@ -324,68 +344,71 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         else
           tma_load_2d(dst, &cmap_tail, c.gg * kCodeBytesPerGroupRow, c.b * prm.tile_rows,
                       &cfull[cs]);
-        issued = j + 1;
       }
-      if (!ok) {
-        fail();
-        for (int k = issued - NC < 0 ? 0 : issued - NC; k < issued; ++k)
-          mbar_wait_bounded(&cfull[k % NC], (k / NC) & 1, prm.drain_ns);
-        for (int k = issued_m - kMetaSlots < 0 ? 0 : issued_m - kMetaSlots; k < issued_m; ++k)
-          mbar_wait_bounded(&mfull[k % kMetaSlots], (k / kMetaSlots) & 1, prm.drain_ns);
-      }
+      __syncwarp();
+      issued = j + 1;
+    }
+    if (!ok) {
+      if (lane == 0) fail();
+      for (int k = issued - NC < 0 ? 0 : issued - NC; k < issued; ++k)
+        warp_wait(&cfull[k % NC], (k / NC) & 1, prm.drain_ns);
+      for (int k = issued_m - kMetaSlots < 0 ? 0 : issued_m - kMetaSlots; k < issued_m; ++k)
+        warp_wait(&mfull[k % kMetaSlots], (k / kMetaSlots) & 1, prm.drain_ns);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ activation producer
-    if (lane == 0) {
-      GroupCursor c;
-      c.init(g, t0);
-      int issued_b = 0, issued_x = 0;
-      bool ok = true;
-      for (int j = 0; j < ngroups; ++j, c.next(g)) {
-        const int bs = j % kBSlots, xs = j % kXsSlots;
-        const int k0 = c.s * kSlabK + c.gg * kGroup;
-        if (j >= kBSlots) ok = mbar_wait_bounded(&bempty[bs], ((j / kBSlots) - 1) & 1, prm.wait_ns);
-        if (!ok || *abort_flag) { ok = false; break; }
+    GroupCursor c;
+    c.init(g, t0);
+    int issued_b = 0, issued_x = 0;
+    bool ok = true;
+    for (int j = 0; j < ngroups; ++j, c.next(g)) {
+      const int bs = j % kBSlots, xs = j % kXsSlots;
+      const int k0 = c.s * kSlabK + c.gg * kGroup;
+      if (j >= kBSlots) ok = warp_wait(&bempty[bs], ((j / kBSlots) - 1) & 1, prm.wait_ns);
+      if (!ok || *abort_flag) { ok = false; break; }
+      if (elect_one()) {
         uint8_t* bdst = smem + SM::kBOff + bs * SM::kB;
         mbar_arrive_expect_tx(&bfull[bs], 2 * MPAD * 128);
         tma_load_2d(bdst, &xmap, k0, 0, &bfull[bs]);
         tma_load_2d(bdst + MPAD * 128, &xmap, k0 + 64, 0, &bfull[bs]);
-        issued_b = j + 1;
-        if (j >= kXsSlots)
-          ok = mbar_wait_bounded(&xsempty[xs], ((j / kXsSlots) - 1) & 1, prm.wait_ns);
-        if (!ok || *abort_flag) { ok = false; break; }
+      }
+      __syncwarp();
+      issued_b = j + 1;
+      if (j >= kXsSlots) ok = warp_wait(&xsempty[xs], ((j / kXsSlots) - 1) & 1, prm.wait_ns);
+      if (!ok || *abort_flag) { ok = false; break; }
+      if (elect_one()) {
         mbar_arrive_expect_tx(&xsfull[xs], MPAD * 4);
         bulk_copy_g2s(smem + SM::kXsOff + xs * SM::kXs,
                       prm.xsum + (size_t)(c.s * kSlabGroups + c.gg) * kGemmPartialM, MPAD * 4,
                       &xsfull[xs]);
-        issued_x = j + 1;
       }
-      if (!ok) {
-        fail();
-        for (int k = issued_b - kBSlots < 0 ? 0 : issued_b - kBSlots; k < issued_b; ++k)
-          mbar_wait_bounded(&bfull[k % kBSlots], (k / kBSlots) & 1, prm.drain_ns);
-        for (int k = issued_x - kXsSlots < 0 ? 0 : issued_x - kXsSlots; k < issued_x; ++k)
-          mbar_wait_bounded(&xsfull[k % kXsSlots], (k / kXsSlots) & 1, prm.drain_ns);
-      }
+      __syncwarp();
+      issued_x = j + 1;
+    }
+    if (!ok) {
+      if (lane == 0) fail();
+      for (int k = issued_b - kBSlots < 0 ? 0 : issued_b - kBSlots; k < issued_b; ++k)
+        warp_wait(&bfull[k % kBSlots], (k / kBSlots) & 1, prm.drain_ns);
+      for (int k = issued_x - kXsSlots < 0 ? 0 : issued_x - kXsSlots; k < issued_x; ++k)
+        warp_wait(&xsfull[k % kXsSlots], (k / kXsSlots) & 1, prm.drain_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int j = 0;
-      bool ok = true;
-      constexpr uint32_t idesc = umma_idesc_bf16<MPAD>();
-      const uint32_t b0 = smem_u32(smem + SM::kBOff);
-      for (; j < ngroups; ++j) {
-        const int ab = j % kABufs, bs = j % kBSlots, acc = j % kAccBufs;
-        ok = mbar_wait_bounded(&afull[ab], (j / kABufs) & 1, prm.wait_ns) &&
-             mbar_wait_bounded(&bfull[bs], (j / kBSlots) & 1, prm.wait_ns) &&
-             (j < kAccBufs ||
-              mbar_wait_bounded(&accempty[acc], ((j / kAccBufs) - 1) & 1, prm.wait_ns));
-        if (!ok || *abort_flag) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t bbase = b0 + bs * SM::kB;
-        const uint32_t ta = tmem_base + ab * 64;
-        const uint32_t td = tmem_base + SM::kAccCol + acc * SM::kAccStride;
+    int j = 0;
+    bool ok = true;
+    constexpr uint32_t idesc = umma_idesc_bf16<MPAD>();
+    const uint32_t b0 = smem_u32(smem + SM::kBOff);
+    for (; j < ngroups; ++j) {
+      const int ab = j % kABufs, bs = j % kBSlots, acc = j % kAccBufs;
+      ok = warp_wait(&afull[ab], (j / kABufs) & 1, prm.wait_ns) &&
+           warp_wait(&bfull[bs], (j / kBSlots) & 1, prm.wait_ns) &&
+           (j < kAccBufs || warp_wait(&accempty[acc], ((j / kAccBufs) - 1) & 1, prm.wait_ns));
+      if (!ok || *abort_flag) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t bbase = b0 + bs * SM::kB;
+      const uint32_t ta = tmem_base + ab * 64;
+      const uint32_t td = tmem_base + SM::kAccCol + acc * SM::kAccStride;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // K = 16 slice kk: 8 columns of A; in B, 64-input block kk / 4 and
@@ -397,12 +420,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         umma_commit(&bempty[bs]);
         umma_commit(&accfull[acc]);
       }
-      if (!ok) {
-        fail();
-        // let the MMAs already issued finish before tensor memory is freed
-        if (j > 0)
-          mbar_wait_bounded(&accfull[(j - 1) % kAccBufs], ((j - 1) / kAccBufs) & 1, prm.drain_ns);
-      }
+      __syncwarp();
+    }
+    if (!ok) {
+      if (lane == 0) fail();
+      // let the MMAs already issued finish before tensor memory is freed
+      if (j > 0)
+        warp_wait(&accfull[(j - 1) % kAccBufs], ((j - 1) / kAccBufs) & 1, prm.drain_ns);
     }
   } else if (warp >= 4 && warp < 4 + kDqWarps) {
     // ------------------------------------------------------------ dequantize
@@ -459,9 +483,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int half = (warp - 12) >> 2;        // columns half*EC .. half*EC+EC-1
     const int m0 = half * EC;
     const int row = q4 * 32 + lane;           // row of the tile (= TMEM lane)
-    float run[EC];
+    float2 run[EC / 2];                       // running sums, columns in pairs
 #pragma unroll
-    for (int m = 0; m < EC; ++m) run[m] = 0.0f;
+    for (int m = 0; m < EC / 2; ++m) run[m] = make_float2(0.0f, 0.0f);
     GroupCursor c;
     c.init(g, t0);
     int piece_s0 = -1;
@@ -516,10 +540,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int cc = 0; cc < kMaxB / 8; ++cc)
           if (b0 + cc * 8 < EC) tmem_ld8(tacc + b0 + cc * 8, d + cc * 8);
         tmem_wait_ld();
+        // run += s16 * (D - (128 + z) * sum(x)), two columns per FFMA2
+        const float2 s2 = make_float2(sc, sc), ncz2 = make_float2(-cz, -cz);
 #pragma unroll
-        for (int m = 0; m < kMaxB; ++m)
-          if (b0 + m < EC)
-            run[b0 + m] = fmaf(sc, fmaf(-cz, xt[b0 + m], d[m]), run[b0 + m]);
+        for (int m = 0; m < kMaxB; m += 4)
+          if (b0 + m < EC) {
+            const float4 x4 = *reinterpret_cast<const float4*>(xt + b0 + m);
+            const float2 t0 = __ffma2_rn(ncz2, make_float2(x4.x, x4.y), make_float2(d[m], d[m + 1]));
+            const float2 t1 =
+                __ffma2_rn(ncz2, make_float2(x4.z, x4.w), make_float2(d[m + 2], d[m + 3]));
+            run[(b0 + m) / 2] = __ffma2_rn(s2, t0, run[(b0 + m) / 2]);
+            run[(b0 + m) / 2 + 1] = __ffma2_rn(s2, t1, run[(b0 + m) / 2 + 1]);
+          }
       }
       tc_fence_before();
       __syncwarp();
@@ -536,13 +568,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (n < g.N) {
 #pragma unroll
             for (int m = 0; m < EC; ++m)
-              if (m0 + m < prm.M) prm.y[(size_t)(m0 + m) * g.N + n] = run[m];
+              if (m0 + m < prm.M)
+                prm.y[(size_t)(m0 + m) * g.N + n] = (m & 1) ? run[m / 2].y : run[m / 2].x;
           }
         } else {
 #pragma unroll
           for (int m = 0; m < EC; ++m)
             if (m0 + m < prm.M)
-              prm.partials[((size_t)piece_s0 * kGemmPartialM + m0 + m) * g.Npad + n] = run[m];
+              prm.partials[((size_t)piece_s0 * kGemmPartialM + m0 + m) * g.Npad + n] =
+                  (m & 1) ? run[m / 2].y : run[m / 2].x;
           __threadfence();
           __syncwarp();
           const long long ub = (long long)b * g.NS;
@@ -570,7 +604,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
 #pragma unroll
-        for (int m = 0; m < EC; ++m) run[m] = 0.0f;
+        for (int m = 0; m < EC / 2; ++m) run[m] = make_float2(0.0f, 0.0f);
         piece_s0 = -1;
       }
       c = nc;
