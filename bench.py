@@ -43,7 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None}
+NCU_TRAFFIC = {"sources_sha256": "ae6901fba59f04aba69bd6ccd46a6aeffdea60649770259e8285ca2b67d029bd",
+               "bytes_per_launch": 124904192 + 4314112}
 
 
 def _args():
@@ -54,6 +55,8 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the offline and other-M legs")
+    ap.add_argument("--case", choices=["gemv_m1", "gemm_m16"], default=None,
+                    help="run one small profiling case (3 launches) and exit")
     return ap.parse_args()
 
 
@@ -235,6 +238,8 @@ def run_ours(a, rank: int, world: int, local_rank: int):
     e2e = run_e2e(a, qw, copies, ncopies, x, M, N, K, sym, dev, stream, ws, ws_bytes, world)
 
     if not a.no_extras:
+        extras["isolated"] = time_isolated(launch, stream, dev, algorithmic_bytes(M, N, K, sym))
+        extras["read_ceiling"] = time_read_ceiling(dev, stream)
         extras["other_m"] = time_other_m(qw, copies, ncopies, N, K, sym, dev, stream)
 
     bytes_per = algorithmic_bytes(M, N, K, sym)
@@ -267,6 +272,12 @@ def run_ours(a, rank: int, world: int, local_rank: int):
         "e2e": e2e,
         "clocks": clocks,
     }
+    if "read_ceiling" in extras:
+        extras["read_ceiling"]["gemv_frac"] = round(achieved_gbs / extras["read_ceiling"]["gbs"], 4)
+    if not a.no_extras:
+        del copies, qw
+        torch.cuda.empty_cache()
+        extras["gemm"] = time_gemm(dev, stream)
     line.update(extras)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(W, x, N, K, sym)
@@ -325,6 +336,115 @@ def time_offline(Wt, qw, stream, N, K, sym):
         res[name] = {"us": round(us, 2), "bytes": nbytes,
                      "gbs": round(nbytes / (us * 1e-6) / 1e9, 1)}
     return res
+
+
+def time_isolated(launch, stream, dev, nbytes, reps=200, warm=20):
+    """Single launches, each after an L2 flush (a 2x-L2 buffer is rewritten
+    outside the timed pair of events): median, p10, p90 in microseconds."""
+    import torch
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    ts = []
+    with torch.cuda.stream(stream):
+        for i in range(warm + reps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            launch(i, stream)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= warm:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+    ts.sort()
+    q = lambda f: ts[min(len(ts) - 1, int(f * len(ts)))]
+    return {"us_median": round(q(0.5), 3), "us_p10": round(q(0.1), 3), "us_p90": round(q(0.9), 3),
+            "gbs_median": round(nbytes / (q(0.5) * 1e-6) / 1e9, 1), "reps": reps,
+            "protocol": "one launch per event pair after a 2xL2 flush, 20 warm-up"}
+
+
+def time_read_ceiling(dev, stream, nbytes=2 << 30, reps=20):
+    """Read-only HBM rate of this GPU: wq_stream_read_probe over a 2 GiB
+    buffer (16-byte streaming loads), best and median of 20."""
+    import torch
+    from post_weight_quantization_wq_b200 import _binding as abi
+    buf = torch.full((nbytes,), 7, dtype=torch.uint8, device=dev)
+    out = torch.zeros(4, dtype=torch.int32, device=dev)
+    ts = []
+    with torch.cuda.stream(stream):
+        for i in range(reps + 3):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            st = abi.wq_stream_read_probe(buf, nbytes, out, stream)
+            e1.record(stream)
+            e1.synchronize()
+            assert st == 0
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1) * 1e-3)
+    ts.sort()
+    del buf
+    return {"gbs": round(nbytes / ts[0] / 1e9, 1), "gbs_median": round(nbytes / ts[len(ts) // 2] / 1e9, 1),
+            "bytes": nbytes, "kernel": "wq_stream_read_probe (16-byte streaming loads, all SMs)"}
+
+
+def time_gemm(dev, stream):
+    """The tensor-core GEMM (wq_gemm_w4a16) at M = 16, 32, 64 on the two
+    batched-decode shapes (28672x8192 and 8192x28672, asymmetric), graphs of
+    back-to-back launches over copies of the packed weight (> L2)."""
+    import numpy as np
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    from post_weight_quantization_wq_b200 import _binding as abi
+    from post_weight_quantization_wq_b200 import inputs
+    out = {}
+    cid = 4
+    wl = inputs.WORKLOADS[cid]
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    for li, lin in enumerate(wl.linears):
+        N, K = lin.N, lin.K
+        W = inputs.workload_weight(cid, li)
+        Wt = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+        del W
+        qw = wq.quantize(Wt, symmetric=wl.sym, stream=stream)
+        torch.cuda.synchronize(dev)
+        del Wt
+        ncopies = max(3, math.ceil(3 * l2 / qw.packed.numel()))
+        copies = [qw.packed] + [qw.packed.clone() for _ in range(ncopies - 1)]
+        for M in wl.Ms:
+            x = inputs.workload_activations(cid, li, M)
+            xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            ws_bytes = abi.wq_workspace_bytes(M, N, K)
+            ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+            def launch(i, s):
+                st = abi.wq_gemm_w4a16(xt, None, copies[i % ncopies], M, N, K, 128, wl.sym, 1, y,
+                                       ws, ws_bytes, s)
+                assert st == 0
+
+            steps = 1000
+            graphs = build_graphs(launch, stream, steps, 50 * ncopies, dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                for g in graphs[:2]:
+                    g.replay()
+                e0.record(stream)
+                for g in graphs:
+                    g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / steps
+            b = algorithmic_bytes(M, N, K, wl.sym)
+            out[f"{N}x{K}_m{M}"] = {"us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1),
+                                    "tflops": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 1),
+                                    "launches": steps + 1}
+        del copies, qw
+        torch.cuda.empty_cache()
+    if abi.wq_last_device_status(stream) != 0:
+        raise RuntimeError("device error in the GEMM leg")
+    return out
 
 
 def time_other_m(qw, copies, ncopies, N, K, sym, dev, stream):
@@ -405,8 +525,11 @@ def run_e2e(a, qw, copies, ncopies, x, M, N, K, sym, dev, stream, ws, ws_bytes, 
 
 
 def cpu_baseline(W, x, N, K, sym, target_s: float = 10.0):
-    """The CPU oracle (single-threaded C, fp64) on a bounded sample of output
-    rows of the same linear, scaled to one full linear."""
+    """The CPU oracle (plain C, fp64) on a bounded sample of output rows of the
+    same linear, scaled to one full linear: once single-threaded, once on all
+    host cores (the unchanged oracle called on disjoint row ranges from one
+    thread per core; the C call releases the GIL)."""
+    import concurrent.futures as cf
     import numpy as np
     import oracle
     rows0 = 64
@@ -422,9 +545,20 @@ def cpu_baseline(W, x, N, K, sym, target_s: float = 10.0):
     t = time.perf_counter()
     oracle.linear(x, P, s, z, K, sym=sym)
     el = time.perf_counter() - t
-    return {"value": round(el / R * N * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+    single = el / R * N * 1e6
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    chunks = [np.arange(i, min(R, i + max(1, R // cores)), dtype=np.int64)
+              for i in range(0, R, max(1, R // cores))]
+    t = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        list(ex.map(lambda r: oracle.linear(x, P, s, z, K, sym=sym, rows=r), chunks))
+    el_mt = time.perf_counter() - t
+    multi = el_mt / R * N * 1e6
+    return {"value": round(multi, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{R} of {N} output rows of the 8192x28672 linear at M=1 (fp64 C oracle, "
-                      f"dequantize + dot per row), {el:.1f} s, scaled to the full linear",
+                      f"dequantize + dot per row) on {cores} threads ({el_mt:.2f} s) and on one "
+                      f"thread ({el:.1f} s), scaled to the full linear",
+            "single_thread_value": round(single, 1),
             "host_cpu": _cpu_model(), "host_cores_available": os.cpu_count()}
 
 
@@ -460,11 +594,11 @@ def run_reference(a, rank: int, world: int):
     rows = [np.array([i], np.int64) for i in range(R)]
     for i in range(a.warmup):
         oracle.linear(x, P, s, z, K, sym=sym, rows=rows[i % R])
-    # bound the run: at most ~120 s of steps
+    # bound the run: at most ~60 s of steps
     t0 = time.perf_counter()
     oracle.linear(x, P, s, z, K, sym=sym, rows=rows[0])
     per = time.perf_counter() - t0
-    steps = min(a.steps, max(1, int(120.0 / max(per, 1e-9))))
+    steps = min(a.steps, max(1, int(60.0 / max(per, 1e-9))))
     t0 = time.perf_counter()
     for i in range(steps):
         oracle.linear(x, P, s, z, K, sym=sym, rows=rows[i % R])
@@ -505,8 +639,35 @@ def max_over_ranks(v, world, dev):
     return float(t.item())
 
 
+def run_case(a):
+    """A few launches of one kernel on one workload, for profilers: gemv_m1 =
+    wq_gemv_w4a16 on 8192x28672 at M = 1; gemm_m16 = wq_gemm_w4a16 on
+    28672x8192 at M = 16 (asymmetric).  About 1 GB on the device."""
+    import numpy as np
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    from post_weight_quantization_wq_b200 import inputs
+    cid, li, M = (WORKLOAD_CID, WORKLOAD_LIN, 1) if a.case == "gemv_m1" else (4, 0, 16)
+    W = inputs.workload_weight(cid, li)
+    x = inputs.workload_activations(cid, li, M)
+    Wt = torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16)
+    del W
+    qw = wq.quantize(Wt, symmetric=inputs.WORKLOADS[cid].sym)
+    del Wt
+    xt = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    for _ in range(3):
+        y = wq.linear(xt, qw)
+    torch.cuda.synchronize()
+    if wq.last_device_status() != 0:
+        raise RuntimeError("device error")
+    print(json.dumps({"case": a.case, "y_sum": float(y.double().sum())}))
+
+
 def main():
     a = _args()
+    if a.case:
+        run_case(a)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -230,6 +230,19 @@ wq_status wq_gemv_w4a16_static(const void* x, const float* inv_act_scale, const 
  */
 void wq_debug_set_wait_limit_ns(unsigned long long ns);
 
+/*
+ * wq_stream_read_probe -- measurement helper with no counterpart on the
+ * quantization pages: read `bytes` bytes of device memory at `buf` once, with
+ * 16-byte streaming loads from every SM, and write their 32-bit XOR checksum
+ * to *out (device pointer, 4-byte aligned; the call zeroes it first).  Timing
+ * it gives the read-only HBM rate of this GPU, the ceiling for the
+ * weight-streaming linears above (which read their weights once and write
+ * almost nothing).  buf 16-byte aligned, bytes a positive multiple of 16
+ * (WQ_ERR_INVALID_ARG / WQ_ERR_MISALIGNED otherwise).  Asynchronous on
+ * `stream`.
+ */
+wq_status wq_stream_read_probe(const void* buf, size_t bytes, uint32_t* out, wq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

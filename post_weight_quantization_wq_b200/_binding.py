@@ -44,6 +44,7 @@ SIGNATURES = {
     "wq_gemv_w4a16_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "wq_last_device_status": (_I, [_P]),
     "wq_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "wq_stream_read_probe": (_I, [_P, _S, _P, _P]),
 }
 
 _lock = threading.Lock()
@@ -149,3 +150,7 @@ def wq_last_device_status(stream=None) -> int:
 
 def wq_debug_set_wait_limit_ns(ns: int) -> None:
     load().wq_debug_set_wait_limit_ns(int(ns))
+
+
+def wq_stream_read_probe(buf, nbytes, out, stream=None) -> int:
+    return load().wq_stream_read_probe(_ptr(buf), int(nbytes), _ptr(out), _stream(stream))

@@ -125,3 +125,13 @@ def test_static_gemv_validation_before_launch():
     assert st == abi.WQ_ERR_UNSUPPORTED_SHAPE
     st = abi.wq_gemv_w4a16_static(0x1004, None, 0x2000, 1, 256, 1024, 128, 0, 1, 0x3000, 0)
     assert st == abi.WQ_ERR_MISALIGNED
+
+
+def test_stream_read_probe_validation_before_launch():
+    # argument errors are reported before any CUDA call (no GPU needed)
+    assert abi.wq_stream_read_probe(None, 1024, 64, 0) == abi.WQ_ERR_INVALID_ARG
+    assert abi.wq_stream_read_probe(256, 0, 64, 0) == abi.WQ_ERR_INVALID_ARG
+    assert abi.wq_stream_read_probe(256, 1000, 64, 0) == abi.WQ_ERR_INVALID_ARG
+    assert abi.wq_stream_read_probe(256, 1024, None, 0) == abi.WQ_ERR_INVALID_ARG
+    assert abi.wq_stream_read_probe(264, 1024, 64, 0) == abi.WQ_ERR_MISALIGNED
+    assert abi.wq_stream_read_probe(256, 1024, 66, 0) == abi.WQ_ERR_MISALIGNED
