@@ -415,7 +415,7 @@ def time_gemm(dev, stream):
             x = inputs.workload_activations(cid, li, M)
             xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
             y = torch.empty((M, N), dtype=torch.float32, device=dev)
-            ws_bytes = abi.wq_workspace_bytes(M, N, K)
+            ws_bytes = abi.wq_gemm_workspace_bytes(M, N, K)
             ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
             def launch(i, s):
@@ -448,39 +448,42 @@ def time_gemm(dev, stream):
 
 
 def time_other_m(qw, copies, ncopies, N, K, sym, dev, stream):
-    """GEMV at M = 2, 4, 8 on the same weight (2000 launches each, graphs)."""
+    """The same weight at M = 2, 4, 8 through the CUDA-core GEMV, and at
+    M = 4, 8 through the tensor-core GEMM (2000 launches each, graphs)."""
     import numpy as np
     import torch
     from post_weight_quantization_wq_b200 import _binding as abi
     from post_weight_quantization_wq_b200 import inputs
     out = {}
-    for M in (2, 4, 8):
-        x = inputs.workload_activations(WORKLOAD_CID, WORKLOAD_LIN, M)
-        xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
-        y = torch.empty((M, N), dtype=torch.float32, device=dev)
-        ws_bytes = abi.wq_workspace_bytes(M, N, K)
-        ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    for path, Ms in (("gemv", (2, 4, 8)), ("gemm", (4, 8))):
+        fn = abi.wq_gemv_w4a16 if path == "gemv" else abi.wq_gemm_w4a16
+        for M in Ms:
+            x = inputs.workload_activations(WORKLOAD_CID, WORKLOAD_LIN, M)
+            xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            ws_bytes = (abi.wq_workspace_bytes if path == "gemv" else abi.wq_gemm_workspace_bytes)(M, N, K)
+            ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
-        def launch(i, s):
-            st = abi.wq_gemv_w4a16(xt, None, copies[i % ncopies], M, N, K, 128, sym, 1, y, ws,
-                                   ws_bytes, s)
-            assert st == 0
+            def launch(i, s):
+                st = fn(xt, None, copies[i % ncopies], M, N, K, 128, sym, 1, y, ws, ws_bytes, s)
+                assert st == 0
 
-        steps = 2000
-        graphs = build_graphs(launch, stream, steps, 100 * ncopies, dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            for g in graphs[:2]:
-                g.replay()
-            e0.record(stream)
-            for g in graphs:
-                g.replay()
-            e1.record(stream)
-        e1.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / steps
-        b = algorithmic_bytes(M, N, K, sym)
-        out[str(M)] = {"us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1)}
+            steps = 2000
+            graphs = build_graphs(launch, stream, steps, 100 * ncopies, dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                for g in graphs[:2]:
+                    g.replay()
+                e0.record(stream)
+                for g in graphs:
+                    g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / steps
+            b = algorithmic_bytes(M, N, K, sym)
+            key = str(M) if path == "gemv" else f"{M}_tensor_cores"
+            out[key] = {"us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1), "entry": fn.__name__}
     return out
 
 

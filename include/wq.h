@@ -140,11 +140,12 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
                          size_t packed_bytes, wq_stream_t stream);
 
 /*
- * wq_workspace_bytes -- workspace needed by wq_gemv_w4a16 (M = 1..8) or
- * wq_gemm_w4a16 (M = 16..64) for these sizes, or 0 when the call needs none
- * (and for M outside both ranges).  It holds completion counters and split-K
- * partial sums; for wq_gemm_w4a16 also the per-group sums of x (so every
- * GEMM call needs one).  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
+ * wq_workspace_bytes -- workspace needed by wq_gemv_w4a16 for M = 1..8
+ * (0 when that call needs none), and by wq_gemm_w4a16 for M = 9..64 (the
+ * only entry point for those M); 0 for M outside 1..64 or invalid sizes.
+ * wq_gemm_workspace_bytes -- workspace needed by wq_gemm_w4a16, M = 1..64.
+ * A workspace holds completion counters and split-K partial sums; the GEMM's
+ * also holds the per-group sums of x, so every GEMM call needs one.  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
  * the counters: they must be zero before the first call that uses a
  * workspace (allocate it zero-filled), and every call that completes leaves
  * them zero again, so one workspace serves any number of later calls of any
@@ -152,6 +153,7 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
  */
 #define WQ_WORKSPACE_COUNTER_BYTES 262144
 size_t wq_workspace_bytes(int M, int N, int K);
+size_t wq_gemm_workspace_bytes(int M, int N, int K);
 
 /*
  * wq_gemv_w4a16 -- the W4A16 decode linear for M = 1..8 activation rows
@@ -174,8 +176,10 @@ wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* p
                         void* workspace, size_t ws_bytes, wq_stream_t stream);
 
 /*
- * wq_gemm_w4a16 -- the same linear for M = 16..64 activation rows on the
- * tensor cores (tcgen05): per group, the weights are dequantized into tensor
+ * wq_gemm_w4a16 -- the same linear for M = 1..64 activation rows on the
+ * tensor cores (tcgen05; the activation tile is zero-padded to 16, 32, 48
+ * or 64 rows, so it pays off from about M = 3, where the CUDA-core GEMV
+ * becomes issue-bound): per group, the weights are dequantized into tensor
  * memory as bf16 tiles holding the exact integers 128 + q, multiplied with x
  * on the tensor cores with fp32 accumulation, and the group's exact
  * contribution s16 * (D - (128 + z) * sum_k x[m][k]) is added in fp32.  Arguments as wq_gemv_w4a16; inv_act_scale must be NULL

@@ -61,10 +61,12 @@ def quantize(W, awq_scale=None, symmetric: bool = False, stream=None,
 _workspaces = {}
 
 
-def workspace_for(M: int, N: int, K: int, device):
-    """A zero-filled workspace large enough for (M, N, K), cached per device."""
+def workspace_for(M: int, N: int, K: int, device, path: str = "gemv"):
+    """A zero-filled workspace large enough for (M, N, K) on the given path,
+    cached per device (it only grows)."""
     import torch
-    need = abi.wq_workspace_bytes(M, N, K)
+    need = abi.wq_gemm_workspace_bytes(M, N, K) if path == "gemm" else \
+        abi.wq_workspace_bytes(M, N, K)
     if need == 0:
         return None, 0
     key = (str(device),)
@@ -75,17 +77,28 @@ def workspace_for(M: int, N: int, K: int, device):
     return ws, ws.numel()
 
 
-def linear(x, qw: QuantizedWeight, inv_act_scale=None, out=None, workspace=None, stream=None):
-    """y = x' dequant(W)^T as fp32 [M][N] for a bf16 CUDA tensor x [M][K]."""
+GEMV_MAX_ROWS = 2
+
+
+def linear(x, qw: QuantizedWeight, inv_act_scale=None, out=None, workspace=None, stream=None,
+           path=None):
+    """y = x' dequant(W)^T as fp32 [M][N] for a bf16 CUDA tensor x [M][K].
+    path: None (choose by M), "gemv" (wq_gemv_w4a16, M <= 8) or "gemm"
+    (wq_gemm_w4a16, tensor cores, no AWQ factor)."""
     import torch
     M, K = x.shape
     assert K == qw.K
     y = out if out is not None else torch.empty((M, qw.N), dtype=torch.float32, device=x.device)
+    # CUDA-core GEMV up to 2 rows (HBM-bound) and for the AWQ fold (its
+    # scaled activations are not exact in a bf16 tensor-core operand);
+    # tensor-core GEMM from 3 rows on, where the GEMV becomes issue-bound
+    if path is None:
+        path = "gemv" if (M <= GEMV_MAX_ROWS or inv_act_scale is not None) else "gemm"
     if workspace is None:
-        ws, ws_bytes = workspace_for(M, qw.N, K, x.device)
+        ws, ws_bytes = workspace_for(M, qw.N, K, x.device, path)
     else:
         ws, ws_bytes = workspace, workspace.numel()
-    fn = abi.wq_gemv_w4a16 if M <= 8 else abi.wq_gemm_w4a16
+    fn = abi.wq_gemv_w4a16 if path == "gemv" else abi.wq_gemm_w4a16
     _check(fn(x, inv_act_scale, qw.packed, M, qw.N, K, GROUP, qw.symmetric, LAYOUT, y, ws,
               ws_bytes, stream), fn.__name__)
     return y

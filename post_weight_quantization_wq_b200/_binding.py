@@ -39,6 +39,7 @@ SIGNATURES = {
     "wq_packed_bytes": (_S, [_I, _I, _I, _I, _I]),
     "wq_pack_layout": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _S, _P]),
     "wq_workspace_bytes": (_S, [_I, _I, _I]),
+    "wq_gemm_workspace_bytes": (_S, [_I, _I, _I]),
     "wq_gemv_w4a16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _S, _P]),
     "wq_gemm_w4a16": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _S, _P]),
     "wq_gemv_w4a16_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -121,6 +122,10 @@ def wq_pack_layout(qweight, scales, zeros, N, K, group_size, symmetric, layout, 
 
 def wq_workspace_bytes(M, N, K) -> int:
     return load().wq_workspace_bytes(M, N, K)
+
+
+def wq_gemm_workspace_bytes(M, N, K) -> int:
+    return load().wq_gemm_workspace_bytes(M, N, K)
 
 
 def wq_gemv_w4a16(x, inv_act_scale, packed, M, N, K, group_size, symmetric, layout, y,

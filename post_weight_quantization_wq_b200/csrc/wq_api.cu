@@ -123,7 +123,7 @@ wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CU
 
 wq_status check_linear(const void* x, const float* inv_s, const void* packed, int M, int Mlo,
                        int Mhi, int N, int K, int group_size, int symmetric, int layout, float* y,
-                       void* workspace, size_t ws_bytes) {
+                       void* workspace, size_t ws_bytes, bool gemm) {
   wq_status st = check_dims(N, K, group_size);
   if (st != WQ_OK) return st;
   if (M < Mlo || M > Mhi) return WQ_ERR_UNSUPPORTED_SHAPE;
@@ -132,7 +132,7 @@ wq_status check_linear(const void* x, const float* inv_s, const void* packed, in
   if (!x || !packed || !y) return WQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(y) || (inv_s && !aligned16(inv_s)))
     return WQ_ERR_MISALIGNED;
-  const size_t need = wq_workspace_bytes(M, N, K);
+  const size_t need = gemm ? wq::gemm_workspace_bytes(M, N, K) : wq::gemv_workspace_bytes(M, N, K);
   if (need > 0) {
     if (!workspace || ws_bytes < need) return WQ_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(workspace)) return WQ_ERR_MISALIGNED;
@@ -223,15 +223,21 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
 size_t wq_workspace_bytes(int M, int N, int K) {
   if (N <= 0 || K <= 0 || K % WQ_GROUP_SIZE || N > WQ_MAX_DIM || K > WQ_MAX_DIM) return 0;
   if (M >= 1 && M <= 8) return wq::gemv_workspace_bytes(M, N, K);
-  if (M >= 16 && M <= 64) return wq::gemm_workspace_bytes(M, N, K);
+  if (M >= 9 && M <= 64) return wq::gemm_workspace_bytes(M, N, K);
   return 0;
+}
+
+size_t wq_gemm_workspace_bytes(int M, int N, int K) {
+  if (N <= 0 || K <= 0 || K % WQ_GROUP_SIZE || N > WQ_MAX_DIM || K > WQ_MAX_DIM) return 0;
+  if (M < 1 || M > 64) return 0;
+  return wq::gemm_workspace_bytes(M, N, K);
 }
 
 wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
                         int N, int K, int group_size, int symmetric, int layout, float* y,
                         void* workspace, size_t ws_bytes, wq_stream_t stream) {
   wq_status st = check_linear(x, inv_act_scale, packed, M, 1, 8, N, K, group_size, symmetric,
-                              layout, y, workspace, ws_bytes);
+                              layout, y, workspace, ws_bytes, false);
   if (st != WQ_OK) return st;
   cudaError_t e;
   DeviceState* d = device_state(&e);
@@ -244,8 +250,8 @@ wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* p
 wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
                         int N, int K, int group_size, int symmetric, int layout, float* y,
                         void* workspace, size_t ws_bytes, wq_stream_t stream) {
-  wq_status st = check_linear(x, inv_act_scale, packed, M, 16, 64, N, K, group_size, symmetric,
-                              layout, y, workspace, ws_bytes);
+  wq_status st = check_linear(x, inv_act_scale, packed, M, 1, 64, N, K, group_size, symmetric,
+                              layout, y, workspace, ws_bytes, true);
   if (st != WQ_OK) return st;
   if (inv_act_scale) return WQ_ERR_INVALID_ARG;
   cudaError_t e;

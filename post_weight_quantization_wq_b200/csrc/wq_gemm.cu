@@ -52,7 +52,7 @@ struct GemmParams {
   const uint8_t* packed;
   const float* xsum;       // fp32 [NG][64]: sum of x over each group, per row of x
   float* y;
-  float* partials;         // fp32 [NS][64][Npad]
+  float* partials;         // fp32 [NS][Mpad][Npad]
   unsigned* counters;
   int* err;
   Geom g;
@@ -69,28 +69,35 @@ constexpr int kGemmWarps = 20;
 constexpr int kGemmThreads = kGemmWarps * 32;
 constexpr int kDqWarps = 8;
 constexpr int kEpiWarps = 8;
-constexpr int kABufs = 4;                   // A operands in tensor memory
-constexpr int kAccBufs = 4;                 // accumulators in tensor memory
-constexpr int kBSlots = 4;                  // bf16 x tiles
-constexpr int kXsSlots = 8;                 // sum(x) rows
+// The pipeline moves stages of kGps consecutive groups (of this CTA's group
+// sequence): one barrier handoff per stage between the roles.  Group j lives
+// in buffer j % 4 (A operand, accumulator, x tile); stage q = j / 2 uses the
+// barrier pair q % 2.
+constexpr int kGps = 2;                     // groups per stage
+constexpr int kPipe = 2;                    // stages in flight between roles
+constexpr int kABufs = kGps * kPipe;        // A operands in tensor memory (4)
+constexpr int kAccBufs = kABufs;            // accumulators in tensor memory
+constexpr int kBSlots = kABufs;             // bf16 x tiles
+constexpr int kXsStages = 4;                // stage slots of sum(x) rows
+constexpr int kXsSlots = kXsStages * kGps;  // sum(x) rows
 constexpr int kMetaSlots = 8;               // per-tile scales (and zeros)
 constexpr int kMetaSlotBytes = kTileRows * kSlabGroups * 4;   // 2 KB
-constexpr int kGemmPartialM = 64;           // workspace row stride (max M)
+constexpr int kXsumRow = 64;                // floats per group in the sum(x) table
 constexpr int kCodeGroupBytes = kTileRows * kCodeBytesPerGroupRow;   // 8 KB
 constexpr uint32_t kTmemCols = 512;
 
 template <int MPAD>
 struct GemmSmem {
-  static constexpr int kCodeSlots = MPAD <= 32 ? 16 : 12;
+  static constexpr int kCodeStages = MPAD <= 32 ? 8 : 6;      // stage slots of codes
+  static constexpr int kCodeSlots = kCodeStages * kGps;
   static constexpr int kB = MPAD * kGroup * 2;                // bf16 x tile
   static constexpr int kBOff = 0;
   static constexpr int kCodeOff = kBOff + kBSlots * kB;
   static constexpr int kXsOff = kCodeOff + kCodeSlots * kCodeGroupBytes;
-  static constexpr int kXs = kGemmPartialM * 4;                // one sum(x) row
+  static constexpr int kXs = kXsumRow * 4;                     // one sum(x) row
   static constexpr int kMetaOff = kXsOff + kXsSlots * kXs;
   static constexpr int kBarOff = kMetaOff + kMetaSlots * kMetaSlotBytes;
-  static constexpr int kNumBars = 2 * kCodeSlots + 2 * kABufs + 2 * kBSlots + 2 * kXsSlots +
-                                  2 * kAccBufs + 2 * kMetaSlots;
+  static constexpr int kNumBars = 2 * kCodeStages + 6 * kPipe + 2 * kXsStages + 2 * kMetaSlots;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                // slack for 1024-B alignment
   // tensor memory columns: A buffers (64 columns = 128 bf16 each), then
@@ -230,23 +237,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                          const __grid_constant__ CUtensorMap cmap_full,
                          const __grid_constant__ CUtensorMap cmap_tail) {
   using SM = GemmSmem<MPAD>;
-  constexpr int NC = SM::kCodeSlots;
+  constexpr int NCS = SM::kCodeStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const Geom g = prm.g;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
-  uint64_t* cfull = bars;                       // [NC] codes of a group landed (TMA)
-  uint64_t* cempty = cfull + NC;                // [NC] codes read (8 dequant warps)
-  uint64_t* afull = cempty + NC;                // [4] A operand stored (8 dequant warps)
-  uint64_t* aempty = afull + kABufs;            // [4] A operand read by the MMAs (commit)
-  uint64_t* bfull = aempty + kABufs;            // [4] x tile landed (TMA)
-  uint64_t* bempty = bfull + kBSlots;           // [4] x tile read by the MMAs (commit)
-  uint64_t* xsfull = bempty + kBSlots;          // [8] sum(x) row landed
-  uint64_t* xsempty = xsfull + kXsSlots;        // [8] sum(x) row read (8 fold warps)
-  uint64_t* accfull = xsempty + kXsSlots;       // [4] accumulator ready (commit)
-  uint64_t* accempty = accfull + kAccBufs;      // [4] accumulator read (8 fold warps)
-  uint64_t* mfull = accempty + kAccBufs;        // [8] metadata of a tile landed
+  uint64_t* cfull = bars;                       // [NCS] codes of a stage landed (TMA)
+  uint64_t* cempty = cfull + NCS;               // [NCS] codes read (8 dequant warps)
+  uint64_t* afull = cempty + NCS;               // [2] A operands stored (8 dequant warps)
+  uint64_t* aempty = afull + kPipe;             // [2] A operands read by the MMAs (commit)
+  uint64_t* bfull = aempty + kPipe;             // [2] x tiles landed (TMA)
+  uint64_t* bempty = bfull + kPipe;             // [2] x tiles read by the MMAs (commit)
+  uint64_t* accfull = bempty + kPipe;           // [2] accumulators ready (commit)
+  uint64_t* accempty = accfull + kPipe;         // [2] accumulators read (8 fold warps)
+  uint64_t* xsfull = accempty + kPipe;          // [4] sum(x) rows landed
+  uint64_t* xsempty = xsfull + kXsStages;       // [4] sum(x) rows read (8 fold warps)
+  uint64_t* mfull = xsempty + kXsStages;        // [8] metadata of a tile landed
   uint64_t* mempty = mfull + kMetaSlots;        // [8] metadata read (8 fold warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mempty + kMetaSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -256,30 +263,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int G = gridDim.x;
   const long long t0 = (long long)blockIdx.x * prm.tiles / G;
   const long long t1 = (long long)(blockIdx.x + 1) * prm.tiles / G;
-  // groups of this CTA's run of tiles
+  // groups of this CTA's run of tiles, and stages of kGps of them
   int ngroups = 0;
   for (long long u = t0; u < t1; ++u) ngroups += slab_groups(g, (int)(u % g.NS));
+  const int nstages = (ngroups + kGps - 1) / kGps;
+  auto stage_groups = [&](int q) { return ngroups - kGps * q < kGps ? ngroups - kGps * q : kGps; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NC; ++i) {
+    for (int i = 0; i < NCS; ++i) {
       mbar_init(&cfull[i], 1);
       mbar_init(&cempty[i], kDqWarps);
     }
-    for (int i = 0; i < kABufs; ++i) {
+    for (int i = 0; i < kPipe; ++i) {
       mbar_init(&afull[i], kDqWarps);
       mbar_init(&aempty[i], 1);
-    }
-    for (int i = 0; i < kBSlots; ++i) {
       mbar_init(&bfull[i], 1);
       mbar_init(&bempty[i], 1);
-    }
-    for (int i = 0; i < kXsSlots; ++i) {
-      mbar_init(&xsfull[i], 1);
-      mbar_init(&xsempty[i], kEpiWarps);
-    }
-    for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&accfull[i], 1);
       mbar_init(&accempty[i], kEpiWarps);
+    }
+    for (int i = 0; i < kXsStages; ++i) {
+      mbar_init(&xsfull[i], 1);
+      mbar_init(&xsempty[i], kEpiWarps);
     }
     for (int i = 0; i < kMetaSlots; ++i) {
       mbar_init(&mfull[i], 1);
@@ -314,44 +319,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     c.init(g, t0);
     int issued = 0, tile = 0, issued_m = 0;
     bool ok = true;
-    for (int j = 0; j < ngroups; ++j, c.next(g)) {
-      if (c.gg == 0) {
-        // the tile's metadata block (128 rows x gs groups) into a meta slot
-        const int ms = tile % kMetaSlots;
-        if (tile >= kMetaSlots)
-          ok = warp_wait(&mempty[ms], ((tile / kMetaSlots) - 1) & 1, prm.wait_ns);
-        if (!ok || *abort_flag) { ok = false; break; }
+    for (int q = 0; q < nstages && ok; ++q) {
+      const int cnt = stage_groups(q);
+      const int cs = q % NCS;
+      if (q >= NCS) ok = warp_wait(&cempty[cs], ((q / NCS) - 1) & 1, prm.wait_ns);
+      if (!ok || *abort_flag) { ok = false; break; }
+      if (elect_one()) mbar_arrive_expect_tx(&cfull[cs], cnt * kCodeGroupBytes);
+      __syncwarp();
+      for (int sub = 0; sub < cnt; ++sub, c.next(g)) {
+        if (c.gg == 0) {
+          // the tile's metadata block (128 rows x gs groups) into a meta slot
+          const int ms = tile % kMetaSlots;
+          if (tile >= kMetaSlots)
+            ok = warp_wait(&mempty[ms], ((tile / kMetaSlots) - 1) & 1, prm.wait_ns);
+          if (!ok || *abort_flag) { ok = false; break; }
+          if (elect_one()) {
+            const uint32_t mbytes = (uint32_t)(kTileRows * c.gs * g.meta);
+            mbar_arrive_expect_tx(&mfull[ms], mbytes);
+            bulk_copy_g2s(smem + SM::kMetaOff + ms * kMetaSlotBytes,
+                          prm.packed + tile_offset(g, c.s, c.b) +
+                              (long long)kTileRows * c.gs * kCodeBytesPerGroupRow,
+                          mbytes, &mfull[ms]);
+          }
+          __syncwarp();
+          issued_m = ++tile;
+        }
         if (elect_one()) {
-          const uint32_t mbytes = (uint32_t)(kTileRows * c.gs * g.meta);
-          mbar_arrive_expect_tx(&mfull[ms], mbytes);
-          bulk_copy_g2s(smem + SM::kMetaOff + ms * kMetaSlotBytes,
-                        prm.packed + tile_offset(g, c.s, c.b) +
-                            (long long)kTileRows * c.gs * kCodeBytesPerGroupRow,
-                        mbytes, &mfull[ms]);
+          uint8_t* dst = smem + SM::kCodeOff + (cs * kGps + sub) * kCodeGroupBytes;
+          if (c.s < prm.ns_full)
+            tma_load_2d(dst, &cmap_full, c.gg * kCodeBytesPerGroupRow,
+                        (c.s * g.NB + c.b) * prm.tile_rows, &cfull[cs]);
+          else
+            tma_load_2d(dst, &cmap_tail, c.gg * kCodeBytesPerGroupRow, c.b * prm.tile_rows,
+                        &cfull[cs]);
         }
         __syncwarp();
-        issued_m = ++tile;
       }
-      const int cs = j % NC;
-      if (j >= NC) ok = warp_wait(&cempty[cs], ((j / NC) - 1) & 1, prm.wait_ns);
-      if (!ok || *abort_flag) { ok = false; break; }
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&cfull[cs], kCodeGroupBytes);
-        uint8_t* dst = smem + SM::kCodeOff + cs * kCodeGroupBytes;
-        if (c.s < prm.ns_full)
-          tma_load_2d(dst, &cmap_full, c.gg * kCodeBytesPerGroupRow,
-                      (c.s * g.NB + c.b) * prm.tile_rows, &cfull[cs]);
-        else
-          tma_load_2d(dst, &cmap_tail, c.gg * kCodeBytesPerGroupRow, c.b * prm.tile_rows,
-                      &cfull[cs]);
-      }
-      __syncwarp();
-      issued = j + 1;
+      issued = q + 1;
     }
     if (!ok) {
       if (lane == 0) fail();
-      for (int k = issued - NC < 0 ? 0 : issued - NC; k < issued; ++k)
-        warp_wait(&cfull[k % NC], (k / NC) & 1, prm.drain_ns);
+      // a stage whose expect_tx was posted but not all its copies issued
+      // never completes; the bounded waits just run out for it
+      for (int k = issued - NCS < 0 ? 0 : issued - NCS; k < issued; ++k)
+        warp_wait(&cfull[k % NCS], (k / NCS) & 1, prm.drain_ns);
       for (int k = issued_m - kMetaSlots < 0 ? 0 : issued_m - kMetaSlots; k < issued_m; ++k)
         warp_wait(&mfull[k % kMetaSlots], (k / kMetaSlots) & 1, prm.drain_ns);
     }
@@ -361,72 +372,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     c.init(g, t0);
     int issued_b = 0, issued_x = 0;
     bool ok = true;
-    for (int j = 0; j < ngroups; ++j, c.next(g)) {
-      const int bs = j % kBSlots, xs = j % kXsSlots;
-      const int k0 = c.s * kSlabK + c.gg * kGroup;
-      if (j >= kBSlots) ok = warp_wait(&bempty[bs], ((j / kBSlots) - 1) & 1, prm.wait_ns);
+    for (int q = 0; q < nstages; ++q) {
+      const int cnt = stage_groups(q);
+      const int ps = q % kPipe, xq = q % kXsStages;
+      if (q >= kPipe) ok = warp_wait(&bempty[ps], ((q / kPipe) - 1) & 1, prm.wait_ns);
+      if (ok && q >= kXsStages)
+        ok = warp_wait(&xsempty[xq], ((q / kXsStages) - 1) & 1, prm.wait_ns);
       if (!ok || *abort_flag) { ok = false; break; }
       if (elect_one()) {
-        uint8_t* bdst = smem + SM::kBOff + bs * SM::kB;
-        mbar_arrive_expect_tx(&bfull[bs], 2 * MPAD * 128);
-        tma_load_2d(bdst, &xmap, k0, 0, &bfull[bs]);
-        tma_load_2d(bdst + MPAD * 128, &xmap, k0 + 64, 0, &bfull[bs]);
+        mbar_arrive_expect_tx(&bfull[ps], cnt * 2 * MPAD * 128);
+        mbar_arrive_expect_tx(&xsfull[xq], cnt * MPAD * 4);
+        GroupCursor cc = c;
+        for (int sub = 0; sub < cnt; ++sub, cc.next(g)) {
+          const int j = kGps * q + sub;
+          const int k0 = cc.s * kSlabK + cc.gg * kGroup;
+          uint8_t* bdst = smem + SM::kBOff + (j % kBSlots) * SM::kB;
+          tma_load_2d(bdst, &xmap, k0, 0, &bfull[ps]);
+          tma_load_2d(bdst + MPAD * 128, &xmap, k0 + 64, 0, &bfull[ps]);
+          bulk_copy_g2s(smem + SM::kXsOff + (xq * kGps + sub) * SM::kXs,
+                        prm.xsum + (size_t)(cc.s * kSlabGroups + cc.gg) * kXsumRow, MPAD * 4,
+                        &xsfull[xq]);
+        }
       }
       __syncwarp();
-      issued_b = j + 1;
-      if (j >= kXsSlots) ok = warp_wait(&xsempty[xs], ((j / kXsSlots) - 1) & 1, prm.wait_ns);
-      if (!ok || *abort_flag) { ok = false; break; }
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&xsfull[xs], MPAD * 4);
-        bulk_copy_g2s(smem + SM::kXsOff + xs * SM::kXs,
-                      prm.xsum + (size_t)(c.s * kSlabGroups + c.gg) * kGemmPartialM, MPAD * 4,
-                      &xsfull[xs]);
-      }
-      __syncwarp();
-      issued_x = j + 1;
+      for (int sub = 0; sub < cnt; ++sub) c.next(g);
+      issued_b = issued_x = q + 1;
     }
     if (!ok) {
       if (lane == 0) fail();
-      for (int k = issued_b - kBSlots < 0 ? 0 : issued_b - kBSlots; k < issued_b; ++k)
-        warp_wait(&bfull[k % kBSlots], (k / kBSlots) & 1, prm.drain_ns);
-      for (int k = issued_x - kXsSlots < 0 ? 0 : issued_x - kXsSlots; k < issued_x; ++k)
-        warp_wait(&xsfull[k % kXsSlots], (k / kXsSlots) & 1, prm.drain_ns);
+      for (int k = issued_b - kPipe < 0 ? 0 : issued_b - kPipe; k < issued_b; ++k)
+        warp_wait(&bfull[k % kPipe], (k / kPipe) & 1, prm.drain_ns);
+      for (int k = issued_x - kXsStages < 0 ? 0 : issued_x - kXsStages; k < issued_x; ++k)
+        warp_wait(&xsfull[k % kXsStages], (k / kXsStages) & 1, prm.drain_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int j = 0;
+    int q = 0;
     bool ok = true;
     constexpr uint32_t idesc = umma_idesc_bf16<MPAD>();
     const uint32_t b0 = smem_u32(smem + SM::kBOff);
-    for (; j < ngroups; ++j) {
-      const int ab = j % kABufs, bs = j % kBSlots, acc = j % kAccBufs;
-      ok = warp_wait(&afull[ab], (j / kABufs) & 1, prm.wait_ns) &&
-           warp_wait(&bfull[bs], (j / kBSlots) & 1, prm.wait_ns) &&
-           (j < kAccBufs || warp_wait(&accempty[acc], ((j / kAccBufs) - 1) & 1, prm.wait_ns));
+    for (; q < nstages; ++q) {
+      const int ps = q % kPipe;
+      ok = warp_wait(&afull[ps], (q / kPipe) & 1, prm.wait_ns) &&
+           warp_wait(&bfull[ps], (q / kPipe) & 1, prm.wait_ns) &&
+           (q < kPipe || warp_wait(&accempty[ps], ((q / kPipe) - 1) & 1, prm.wait_ns));
       if (!ok || *abort_flag) { ok = false; break; }
       tc_fence_after();
-      const uint32_t bbase = b0 + bs * SM::kB;
-      const uint32_t ta = tmem_base + ab * 64;
-      const uint32_t td = tmem_base + SM::kAccCol + acc * SM::kAccStride;
+      const int cnt = stage_groups(q);
       if (elect_one()) {
+        for (int sub = 0; sub < cnt; ++sub) {
+          const int bj = (kGps * q + sub) % kABufs;
+          const uint32_t bbase = b0 + bj * SM::kB;
+          const uint32_t ta = tmem_base + bj * 64;
+          const uint32_t td = tmem_base + SM::kAccCol + bj * SM::kAccStride;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // K = 16 slice kk: 8 columns of A; in B, 64-input block kk / 4 and
-          // a 32-byte step inside its swizzled rows
-          const uint64_t bd = umma_desc_sw128(bbase + (kk >> 2) * (MPAD * 128) + (kk & 3) * 32);
-          umma_bf16_ts(td, ta + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            // K = 16 slice kk: 8 columns of A; in B, 64-input block kk / 4 and
+            // a 32-byte step inside its swizzled rows
+            const uint64_t bd = umma_desc_sw128(bbase + (kk >> 2) * (MPAD * 128) + (kk & 3) * 32);
+            umma_bf16_ts(td, ta + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+          }
         }
-        umma_commit(&aempty[ab]);
-        umma_commit(&bempty[bs]);
-        umma_commit(&accfull[acc]);
+        umma_commit(&aempty[ps]);
+        umma_commit(&bempty[ps]);
+        umma_commit(&accfull[ps]);
       }
       __syncwarp();
     }
     if (!ok) {
       if (lane == 0) fail();
       // let the MMAs already issued finish before tensor memory is freed
-      if (j > 0)
-        warp_wait(&accfull[(j - 1) % kAccBufs], ((j - 1) / kAccBufs) & 1, prm.drain_ns);
+      if (q > 0) warp_wait(&accfull[(q - 1) % kPipe], ((q - 1) / kPipe) & 1, prm.drain_ns);
     }
   } else if (warp >= 4 && warp < 4 + kDqWarps) {
     // ------------------------------------------------------------ dequantize
@@ -441,39 +457,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int off0 = r * 64 + (((2 * h) ^ sw) << 4);
     const int off1 = r * 64 + (((2 * h + 1) ^ sw) << 4);
     bool ok = true;
-    for (int j = 0; j < ngroups; ++j) {
-      const int cs = j % NC, ab = j % kABufs;
-      bool w_ok = mbar_wait_bounded(&cfull[cs], (j / NC) & 1, prm.wait_ns);
-      if (w_ok && j >= kABufs)
-        w_ok = mbar_wait_bounded(&aempty[ab], ((j / kABufs) - 1) & 1, prm.wait_ns);
+    for (int q = 0; q < nstages; ++q) {
+      const int cs = q % NCS, ps = q % kPipe;
+      bool w_ok = mbar_wait_bounded(&cfull[cs], (q / NCS) & 1, prm.wait_ns);
+      if (w_ok && q >= kPipe)
+        w_ok = mbar_wait_bounded(&aempty[ps], ((q / kPipe) - 1) & 1, prm.wait_ns);
       if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
       tc_fence_after();
-      const uint8_t* slot = smem + SM::kCodeOff + cs * kCodeGroupBytes;
-      const uint4 c0 = *reinterpret_cast<const uint4*>(slot + off0);
-      const uint4 c1 = *reinterpret_cast<const uint4*>(slot + off1);
-      const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const int cnt = stage_groups(q);
+      for (int sub = 0; sub < cnt; ++sub) {
+        const int bj = (kGps * q + sub) % kABufs;
+        const uint8_t* slot = smem + SM::kCodeOff + (cs * kGps + sub) * kCodeGroupBytes;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(slot + off0);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(slot + off1);
+        const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t v[16];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          // word covers 8 inputs; slot t of the interleaved word holds input
-          // 2t (t < 4) or 2(t-4)+1, so each LOP3 yields one bf16 pair
-          // (128 + q_even, 128 + q_odd)
-          const uint32_t w = wds[4 * half + q];
-          v[4 * q + 0] = and_or3(w, mlo, b128);
-          v[4 * q + 1] = and_or3(w >> 4, mlo, b128);
-          v[4 * q + 2] = and_or3(w >> 8, mlo, b128);
-          v[4 * q + 3] = and_or3(w >> 12, mlo, b128);
+          for (int qq = 0; qq < 4; ++qq) {
+            // word covers 8 inputs; slot t of the interleaved word holds input
+            // 2t (t < 4) or 2(t-4)+1, so each LOP3 yields one bf16 pair
+            // (128 + q_even, 128 + q_odd)
+            const uint32_t w = wds[4 * half + qq];
+            v[4 * qq + 0] = and_or3(w, mlo, b128);
+            v[4 * qq + 1] = and_or3(w >> 4, mlo, b128);
+            v[4 * qq + 2] = and_or3(w >> 8, mlo, b128);
+            v[4 * qq + 3] = and_or3(w >> 12, mlo, b128);
+          }
+          tmem_st16(lane_base + bj * 64 + half * 16, v);
         }
-        tmem_st16(lane_base + ab * 64 + half * 16, v);
       }
       __syncwarp();                           // every lane's codes are in registers
       if (lane == 0) mbar_arrive(&cempty[cs]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[ab]);
+      if (lane == 0) mbar_arrive(&afull[ps]);
     }
     if (!ok && lane == 0) fail();
   } else if (warp >= 12) {
@@ -492,122 +512,131 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     float scs[kSlabGroups], czs[kSlabGroups];   // this row's (scale, 128 + zero) per group
     int tile = 0;
-    for (int j = 0; j < ngroups; ++j) {
-      const int xs = j % kXsSlots, acc = j % kAccBufs;
-      if (piece_s0 < 0) piece_s0 = c.s;
-      if (c.gg == 0) {
-        // the tile's scales (and zeros) for this row, then release the slot
-        const int ms = tile % kMetaSlots;
-        const bool m_ok = mbar_wait_bounded(&mfull[ms], (tile / kMetaSlots) & 1, prm.wait_ns);
-        if (!__all_sync(0xFFFFFFFFu, m_ok) || *abort_flag) { ok = false; break; }
-        const uint8_t* mb = smem + SM::kMetaOff + ms * kMetaSlotBytes;
-#pragma unroll
-        for (int q = 0; q < kSlabGroups; ++q) {
-          if (q < c.gs) {
-            if (g.sym) {
-              scs[q] = __half2float(reinterpret_cast<const __half*>(mb)[row * c.gs + q]);
-              czs[q] = 136.0f;                 // 128 + 8
-            } else {
-              const __half2 sz = reinterpret_cast<const __half2*>(mb)[row * c.gs + q];
-              scs[q] = __low2float(sz);
-              czs[q] = 128.0f + __high2float(sz);
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&mempty[ms]);
-        ++tile;
-      }
-      float sc = scs[0], cz = czs[0];
-#pragma unroll
-      for (int q = 1; q < kSlabGroups; ++q)
-        if (c.gg == q) { sc = scs[q]; cz = czs[q]; }
-      GroupCursor nc = c;
-      const bool tile_end = nc.next(g);
-      bool w_ok = mbar_wait_bounded(&xsfull[xs], (j / kXsSlots) & 1, prm.wait_ns) &&
-                  mbar_wait_bounded(&accfull[acc], (j / kAccBufs) & 1, prm.wait_ns);
+    for (int q = 0; q < nstages && ok; ++q) {
+      const int ps = q % kPipe, xq = q % kXsStages;
+      bool w_ok = mbar_wait_bounded(&xsfull[xq], (q / kXsStages) & 1, prm.wait_ns) &&
+                  mbar_wait_bounded(&accfull[ps], (q / kPipe) & 1, prm.wait_ns);
       if (!__all_sync(0xFFFFFFFFu, w_ok) || *abort_flag) { ok = false; break; }
       tc_fence_after();
-      const float* xt = reinterpret_cast<const float*>(smem + SM::kXsOff + xs * SM::kXs) + m0;
-      const uint32_t tacc = tmem_base + ((uint32_t)(q4 * 32) << 16) + SM::kAccCol +
-                            acc * SM::kAccStride + m0;
-      // batches of up to 16 columns: load, wait, fold (bounds live registers)
+      const int cnt = stage_groups(q);
+      for (int sub = 0; sub < cnt; ++sub) {
+        const int j = kGps * q + sub;
+        if (piece_s0 < 0) piece_s0 = c.s;
+        if (c.gg == 0) {
+          // the tile's scales (and zeros) for this row, then release the slot
+          const int ms = tile % kMetaSlots;
+          const bool m_ok = mbar_wait_bounded(&mfull[ms], (tile / kMetaSlots) & 1, prm.wait_ns);
+          if (!__all_sync(0xFFFFFFFFu, m_ok) || *abort_flag) { ok = false; break; }
+          const uint8_t* mb = smem + SM::kMetaOff + ms * kMetaSlotBytes;
 #pragma unroll
-      for (int b0 = 0; b0 < EC; b0 += 16) {
-        constexpr int kMaxB = EC < 16 ? EC : 16;
-        float d[kMaxB];
-#pragma unroll
-        for (int cc = 0; cc < kMaxB / 8; ++cc)
-          if (b0 + cc * 8 < EC) tmem_ld8(tacc + b0 + cc * 8, d + cc * 8);
-        tmem_wait_ld();
-        // run += s16 * (D - (128 + z) * sum(x)), two columns per FFMA2
-        const float2 s2 = make_float2(sc, sc), ncz2 = make_float2(-cz, -cz);
-#pragma unroll
-        for (int m = 0; m < kMaxB; m += 4)
-          if (b0 + m < EC) {
-            const float4 x4 = *reinterpret_cast<const float4*>(xt + b0 + m);
-            const float2 t0 = __ffma2_rn(ncz2, make_float2(x4.x, x4.y), make_float2(d[m], d[m + 1]));
-            const float2 t1 =
-                __ffma2_rn(ncz2, make_float2(x4.z, x4.w), make_float2(d[m + 2], d[m + 3]));
-            run[(b0 + m) / 2] = __ffma2_rn(s2, t0, run[(b0 + m) / 2]);
-            run[(b0 + m) / 2 + 1] = __ffma2_rn(s2, t1, run[(b0 + m) / 2 + 1]);
+          for (int qq = 0; qq < kSlabGroups; ++qq) {
+            if (qq < c.gs) {
+              if (g.sym) {
+                scs[qq] = __half2float(reinterpret_cast<const __half*>(mb)[row * c.gs + qq]);
+                czs[qq] = 136.0f;              // 128 + 8
+              } else {
+                const __half2 sz = reinterpret_cast<const __half2*>(mb)[row * c.gs + qq];
+                scs[qq] = __low2float(sz);
+                czs[qq] = 128.0f + __high2float(sz);
+              }
+            }
           }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[acc]);
-      if (lane == 0) mbar_arrive(&xsempty[xs]);
-      if (!tile_end) { c = nc; continue; }
-      // ---- last group of a tile: end of this CTA's piece of row tile b?
-      const bool piece_end = (c.s == g.NS - 1) || (j == ngroups - 1);
-      if (piece_end) {
-        const int b = c.b;
-        const bool whole = (piece_s0 == 0) && (c.s == g.NS - 1);
-        const int n = b * kTileRows + row;
-        if (whole) {
-          if (n < g.N) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&mempty[ms]);
+          ++tile;
+        }
+        float sc = scs[0], cz = czs[0];
+#pragma unroll
+        for (int qq = 1; qq < kSlabGroups; ++qq)
+          if (c.gg == qq) { sc = scs[qq]; cz = czs[qq]; }
+        GroupCursor nc = c;
+        const bool tile_end = nc.next(g);
+        const float* xt =
+            reinterpret_cast<const float*>(smem + SM::kXsOff + (xq * kGps + sub) * SM::kXs) + m0;
+        const uint32_t tacc = tmem_base + ((uint32_t)(q4 * 32) << 16) + SM::kAccCol +
+                              (j % kAccBufs) * SM::kAccStride + m0;
+        // batches of up to 16 columns: load, wait, fold (bounds live registers)
+#pragma unroll
+        for (int b0 = 0; b0 < EC; b0 += 16) {
+          constexpr int kMaxB = EC < 16 ? EC : 16;
+          float d[kMaxB];
+#pragma unroll
+          for (int cc = 0; cc < kMaxB / 8; ++cc)
+            if (b0 + cc * 8 < EC) tmem_ld8(tacc + b0 + cc * 8, d + cc * 8);
+          tmem_wait_ld();
+          // run += s16 * (D - (128 + z) * sum(x)), two columns per FFMA2
+          const float2 s2 = make_float2(sc, sc), ncz2 = make_float2(-cz, -cz);
+#pragma unroll
+          for (int m = 0; m < kMaxB; m += 4)
+            if (b0 + m < EC) {
+              const float4 x4 = *reinterpret_cast<const float4*>(xt + b0 + m);
+              const float2 t0v =
+                  __ffma2_rn(ncz2, make_float2(x4.x, x4.y), make_float2(d[m], d[m + 1]));
+              const float2 t1v =
+                  __ffma2_rn(ncz2, make_float2(x4.z, x4.w), make_float2(d[m + 2], d[m + 3]));
+              run[(b0 + m) / 2] = __ffma2_rn(s2, t0v, run[(b0 + m) / 2]);
+              run[(b0 + m) / 2 + 1] = __ffma2_rn(s2, t1v, run[(b0 + m) / 2 + 1]);
+            }
+        }
+        if (!tile_end) { c = nc; continue; }
+        // ---- last group of a tile: end of this CTA's piece of row tile b?
+        const bool piece_end = (c.s == g.NS - 1) || (j == ngroups - 1);
+        if (piece_end) {
+          const int b = c.b;
+          const bool whole = (piece_s0 == 0) && (c.s == g.NS - 1);
+          const int n = b * kTileRows + row;
+          if (whole) {
+            if (n < g.N) {
+#pragma unroll
+              for (int m = 0; m < EC; ++m)
+                if (m0 + m < prm.M)
+                  prm.y[(size_t)(m0 + m) * g.N + n] = (m & 1) ? run[m / 2].y : run[m / 2].x;
+            }
+          } else {
 #pragma unroll
             for (int m = 0; m < EC; ++m)
               if (m0 + m < prm.M)
-                prm.y[(size_t)(m0 + m) * g.N + n] = (m & 1) ? run[m / 2].y : run[m / 2].x;
-          }
-        } else {
-#pragma unroll
-          for (int m = 0; m < EC; ++m)
-            if (m0 + m < prm.M)
-              prm.partials[((size_t)piece_s0 * kGemmPartialM + m0 + m) * g.Npad + n] =
-                  (m & 1) ? run[m / 2].y : run[m / 2].x;
-          __threadfence();
-          __syncwarp();
-          const long long ub = (long long)b * g.NS;
-          const int c_first = owner_of(ub, prm.tiles, G);
-          const int c_last = owner_of(ub + g.NS - 1, prm.tiles, G);
-          unsigned prev = 0;
-          unsigned* ctr =
-              prm.counters + (size_t)b * (kTileRows / kRowsPerCounter) + q4 + 4 * half;
-          if (lane == 0) prev = atomicAdd(ctr, 1u);
-          prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-          if (prev == (unsigned)(c_last - c_first)) {
+                prm.partials[((size_t)piece_s0 * MPAD + m0 + m) * g.Npad + n] =
+                    (m & 1) ? run[m / 2].y : run[m / 2].x;
             __threadfence();
-            const int m_end = prm.M < m0 + EC ? prm.M : m0 + EC;
-            if (n < g.N)
-              for (int m = m0; m < m_end; ++m) {
-                float tot = 0.0f;
-                for (int c2 = c_first; c2 <= c_last; ++c2) {
-                  const long long tc = (long long)c2 * prm.tiles / G;
-                  const int sa = (int)((tc > ub ? tc : ub) - ub);
-                  tot += __ldcg(prm.partials + ((size_t)sa * kGemmPartialM + m) * g.Npad + n);
+            __syncwarp();
+            const long long ub = (long long)b * g.NS;
+            const int c_first = owner_of(ub, prm.tiles, G);
+            const int c_last = owner_of(ub + g.NS - 1, prm.tiles, G);
+            unsigned prev = 0;
+            unsigned* ctr =
+                prm.counters + (size_t)b * (kTileRows / kRowsPerCounter) + q4 + 4 * half;
+            if (lane == 0) prev = atomicAdd(ctr, 1u);
+            prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+            if (prev == (unsigned)(c_last - c_first)) {
+              __threadfence();
+              const int m_end = prm.M < m0 + EC ? prm.M : m0 + EC;
+              if (n < g.N)
+                for (int m = m0; m < m_end; ++m) {
+                  float tot = 0.0f;
+                  for (int c2 = c_first; c2 <= c_last; ++c2) {
+                    const long long tc = (long long)c2 * prm.tiles / G;
+                    const int sa = (int)((tc > ub ? tc : ub) - ub);
+                    tot += __ldcg(prm.partials + ((size_t)sa * MPAD + m) * g.Npad + n);
+                  }
+                  prm.y[(size_t)m * g.N + n] = tot;
                 }
-                prm.y[(size_t)m * g.N + n] = tot;
-              }
-            if (lane == 0) *ctr = 0u;
+              if (lane == 0) *ctr = 0u;
+            }
           }
-        }
 #pragma unroll
-        for (int m = 0; m < EC / 2; ++m) run[m] = make_float2(0.0f, 0.0f);
-        piece_s0 = -1;
+          for (int m = 0; m < EC / 2; ++m) run[m] = make_float2(0.0f, 0.0f);
+          piece_s0 = -1;
+        }
+        c = nc;
       }
-      c = nc;
+      if (!ok) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&accempty[ps]);
+        mbar_arrive(&xsempty[xq]);
+      }
     }
     if (!ok && lane == 0) fail();
   }
@@ -631,7 +660,7 @@ __global__ void __launch_bounds__(256) gemm_xsum_kernel(const uint16_t* __restri
   const int lane = threadIdx.x & 31;
   const int NG = K / kGroup;
   if (warp >= NG) return;
-  for (int m = lane; m < kGemmPartialM; m += 32) {
+  for (int m = lane; m < kXsumRow; m += 32) {
     float acc = 0.0f;
     if (m < M) {
       const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)m * K + warp * kGroup);
@@ -644,21 +673,23 @@ __global__ void __launch_bounds__(256) gemm_xsum_kernel(const uint16_t* __restri
           acc += __uint_as_float(w4[h] << 16) + __uint_as_float(w4[h] & 0xFFFF0000u);
       }
     }
-    xsum[(size_t)warp * kGemmPartialM + m] = acc;
+    xsum[(size_t)warp * kXsumRow + m] = acc;
   }
 }
 
 // ------------------------------------------------------------------ launcher
 
-static size_t gemm_partials_bytes(const Geom& g) {
-  return g.NS <= 1 ? 0 : (size_t)g.NS * kGemmPartialM * g.Npad * sizeof(float);
+static int gemm_mpad(int M) { return (M + 15) / 16 * 16; }
+
+// split-K partial sums: fp32 [NS][Mpad][Npad]
+static size_t gemm_partials_bytes(const Geom& g, int M) {
+  return g.NS <= 1 ? 0 : (size_t)g.NS * gemm_mpad(M) * g.Npad * sizeof(float);
 }
 
 size_t gemm_workspace_bytes(int M, int N, int K) {
-  (void)M;
   const Geom g = make_geom(N, K, 1);
-  return (size_t)kCounterBytes + gemm_partials_bytes(g) +
-         (size_t)g.NG * kGemmPartialM * sizeof(float);
+  return (size_t)kCounterBytes + gemm_partials_bytes(g, M) +
+         (size_t)g.NG * kXsumRow * sizeof(float);
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -746,7 +777,7 @@ cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, 
   prm.counters = static_cast<unsigned*>(workspace);
   prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
   float* xsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes +
-                                         gemm_partials_bytes(prm.g));
+                                         gemm_partials_bytes(prm.g, M));
   prm.xsum = xsum;
   prm.err = err;
   prm.M = M;
@@ -765,8 +796,7 @@ cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const int mpad = (M + 15) / 16 * 16;
-  switch (mpad) {
+  switch (gemm_mpad(M)) {
     case 16: return launch_gemm_t<16>(prm, x, num_sms, stream);
     case 32: return launch_gemm_t<32>(prm, x, num_sms, stream);
     case 48: return launch_gemm_t<48>(prm, x, num_sms, stream);

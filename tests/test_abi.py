@@ -49,13 +49,24 @@ def test_packed_bytes_matches_layout_definition():
 
 
 def test_workspace_bytes():
-    # single slab: no split-K, no workspace
+    C = abi.WQ_WORKSPACE_COUNTER_BYTES
+    # GEMV (M <= 8): one slab needs no workspace; 8192 x 28672 has 56 slabs
+    # and partials for 4 padded rows of x at M = 3
     assert abi.wq_workspace_bytes(1, 4096, 512) == 0
-    n = abi.wq_workspace_bytes(1, 8192, 28672)
-    assert n == abi.WQ_WORKSPACE_COUNTER_BYTES + 56 * 1 * 8192 * 4
-    assert abi.wq_workspace_bytes(3, 8192, 28672) == abi.WQ_WORKSPACE_COUNTER_BYTES + 56 * 4 * 8192 * 4
-    assert abi.wq_workspace_bytes(9, 8192, 8192) == 0          # M between the two paths
-    assert abi.wq_workspace_bytes(16, 8192, 8192) > 0
+    assert abi.wq_workspace_bytes(1, 8192, 28672) == C + 56 * 1 * 8192 * 4
+    assert abi.wq_workspace_bytes(3, 8192, 28672) == C + 56 * 4 * 8192 * 4
+    # GEMM: counters, partials padded to 16-row multiples, sum(x) per group
+    gemm16 = C + 56 * 16 * 8192 * 4 + 224 * 64 * 4
+    assert abi.wq_gemm_workspace_bytes(1, 4096, 512) == C + 4 * 64 * 4
+    assert abi.wq_gemm_workspace_bytes(1, 8192, 28672) == gemm16
+    assert abi.wq_gemm_workspace_bytes(16, 8192, 28672) == gemm16
+    assert abi.wq_gemm_workspace_bytes(17, 8192, 28672) == C + 56 * 32 * 8192 * 4 + 224 * 64 * 4
+    assert abi.wq_workspace_bytes(9, 8192, 28672) == gemm16         # M = 9..64: GEMM only
+    assert abi.wq_workspace_bytes(64, 8192, 28672) == abi.wq_gemm_workspace_bytes(64, 8192, 28672)
+    assert abi.wq_workspace_bytes(0, 8192, 8192) == 0
+    assert abi.wq_workspace_bytes(65, 8192, 8192) == 0
+    assert abi.wq_gemm_workspace_bytes(65, 8192, 8192) == 0
+    assert abi.wq_workspace_bytes(1, 8192, 100) == 0          # K not a multiple of 128
 
 
 @pytest.mark.parametrize("args,expect", [
@@ -80,7 +91,7 @@ def test_quantize_validation_before_launch(args, expect):
 
 
 @pytest.mark.parametrize("fn,M", [("wq_gemv_w4a16", 0), ("wq_gemv_w4a16", 9),
-                                  ("wq_gemm_w4a16", 8), ("wq_gemm_w4a16", 65)])
+                                  ("wq_gemm_w4a16", 0), ("wq_gemm_w4a16", 65)])
 def test_linear_rejects_m_out_of_range(fn, M):
     st = getattr(abi, fn)(0x1000, None, 0x2000, M, 256, 1024, 128, 0, 1, 0x3000, 0x4000,
                           1 << 30, 0)

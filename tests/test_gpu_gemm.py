@@ -1,4 +1,4 @@
-"""GPU W4A16 skinny GEMM (M = 16..64, tcgen05 tensor cores) against the CPU
+"""GPU W4A16 skinny GEMM (M = 1..64, tcgen05 tensor cores) against the CPU
 oracle's fp64 linear: rel-L2 <= 1e-3 and max-abs <= 1e-2 * rms(y)."""
 import numpy as np
 import pytest
@@ -16,10 +16,10 @@ pytestmark = pytest.mark.gpu
 def test_gemm_small(N, K, sym):
     W = inputs.weights(N, K, 0.02, seed=3 * N + K)
     qw, P, s, z = quantize_and_check(W, None, sym)
-    for M in (16, 24, 32, 40, 48, 64):
+    for M in (1, 3, 8, 16, 24, 32, 40, 48, 64):
         chans = inputs.outlier_channels(K, 0.01, seed=K)
         x = inputs.activations(M, K, seed=M + 7 * K, channels=chans, mult=30.0)
-        y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+        y = wq.linear(dev_bf16(x), qw, path="gemm").cpu().numpy()
         check_close(y, oracle.linear(x, P, s, z, K, sym=sym), f"N={N} K={K} M={M}")
 
 
@@ -31,7 +31,7 @@ def test_gemm_zero_point_outside_code_range():
     W = inputs.to_bf16_bits(w)
     qw, P, s, z = quantize_and_check(W, None, False)
     x = inputs.activations(32, K, seed=5)
-    y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+    y = wq.linear(dev_bf16(x), qw, path="gemm").cpu().numpy()
     check_close(y, oracle.linear(x, P, s, z, K, sym=False))
 
 
@@ -40,7 +40,7 @@ def test_gemm_row_tile_split_across_many_ctas():
     W = inputs.weights(N, K, 0.015, seed=21)
     qw, P, s, z = quantize_and_check(W, None, False)
     x = inputs.activations(16, K, seed=22)
-    y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+    y = wq.linear(dev_bf16(x), qw, path="gemm").cpu().numpy()
     check_close(y, oracle.linear(x, P, s, z, K, sym=False))
 
 
@@ -50,7 +50,7 @@ def test_gemm_deterministic():
     W = inputs.weights(N, K, 0.015, seed=31)
     qw, *_ = quantize_and_check(W, None, False)
     x = dev_bf16(inputs.activations(64, K, seed=32))
-    assert torch.equal(wq.linear(x, qw), wq.linear(x, qw))
+    assert torch.equal(wq.linear(x, qw, path="gemm"), wq.linear(x, qw, path="gemm"))
 
 
 @pytest.mark.parametrize("li", [0, 1])
@@ -66,6 +66,6 @@ def test_workload_batched_decode_full_size(li):
     rows = sample_rows(lin.N, seed=40 + li)
     for M in wl.Ms:
         x = inputs.workload_activations(cid, li, M)
-        y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+        y = wq.linear(dev_bf16(x), qw, path="gemm").cpu().numpy()
         yref = oracle.linear(x, P, s, z, lin.K, sym=wl.sym, rows=rows)
         check_close(y[:, rows], yref, f"cfg4 {lin.name} M={M}")

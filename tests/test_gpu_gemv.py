@@ -19,7 +19,7 @@ def test_gemv_small_all_m(N, K, sym):
     qw, P, s, z = quantize_and_check(W, None, sym)
     for M in range(1, 9):
         x = inputs.activations(M, K, seed=M * 31 + K)
-        y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+        y = wq.linear(dev_bf16(x), qw, path="gemv").cpu().numpy()
         yref = oracle.linear(x, P, s, z, K, sym=sym)
         check_close(y, yref, f"N={N} K={K} M={M}")
 
@@ -32,7 +32,7 @@ def test_gemv_row_tile_split_across_many_ctas(M):
     W = inputs.weights(N, K, 0.015, seed=7)
     qw, P, s, z = quantize_and_check(W, None, False)
     x = inputs.activations(M, K, seed=8)
-    y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+    y = wq.linear(dev_bf16(x), qw, path="gemv").cpu().numpy()
     check_close(y, oracle.linear(x, P, s, z, K, sym=False))
 
 
@@ -46,7 +46,7 @@ def test_gemv_awq_fold_small(M):
     qw, P, sc, z = quantize_and_check(W, s, False)
     x = inputs.activations(M, K, seed=94, channels=chans, mult=50.0)
     inv = (1.0 / s).astype(np.float32)
-    y = wq.linear(dev_bf16(x), qw, inv_act_scale=dev_f32(inv)).cpu().numpy()
+    y = wq.linear(dev_bf16(x), qw, inv_act_scale=dev_f32(inv), path="gemv").cpu().numpy()
     yref = oracle.linear(x, P, sc, z, K, sym=False, awq_s=s)
     check_close(y, yref, f"awq M={M}")
 
@@ -58,7 +58,7 @@ def test_gemv_nonfinite_group_gives_nan_rows():
     W = inputs.to_bf16_bits(w)
     qw, P, s, z = quantize_and_check(W, None, False)
     x = inputs.activations(1, K, seed=3)
-    y = wq.linear(dev_bf16(x), qw).cpu().numpy()
+    y = wq.linear(dev_bf16(x), qw, path="gemv").cpu().numpy()
     yref = oracle.linear(x, P, s, z, K, sym=False)
     assert np.isnan(y[0, 9]) and np.isnan(yref[0, 9])
     keep = np.arange(N) != 9
@@ -76,8 +76,8 @@ def test_gemv_deterministic_and_workspace_reuse():
         W = inputs.weights(N, K, 0.02, seed=N + 3 * K)
         qw, P, s, z = quantize_and_check(W, None, False)
         x = dev_bf16(inputs.activations(M, K, seed=K + M))
-        y1 = wq.linear(x, qw, workspace=ws)
-        y2 = wq.linear(x, qw, workspace=ws)
+        y1 = wq.linear(x, qw, workspace=ws, path="gemv")
+        y2 = wq.linear(x, qw, workspace=ws, path="gemv")
         assert torch.equal(y1, y2)
         yref = oracle.linear(x.cpu().view(torch.int16).numpy().view(np.uint16), P, s, z, K,
                              sym=False)
@@ -106,6 +106,6 @@ def test_workload_full_size(cid, li):
     rows = sample_rows(lin.N, seed=cid * 10 + li)
     for M in wl.Ms:
         x = inputs.workload_activations(cid, li, M)
-        y = wq.linear(dev_bf16(x), qw, inv_act_scale=inv).cpu().numpy()
+        y = wq.linear(dev_bf16(x), qw, inv_act_scale=inv, path="gemv").cpu().numpy()
         yref = oracle.linear(x, P, s, z, lin.K, sym=wl.sym, awq_s=s_awq, rows=rows)
         check_close(y[:, rows], yref, f"cfg{cid} {lin.name} M={M}")
