@@ -356,7 +356,6 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
       const int rs = i % RAWS;
       bool ok = true;
       if (i >= STAGES) ok = mbar_wait_bounded(&empty_bar[st], ((i / STAGES) - 1) & 1, prm.wait_ns);
-      if (ok) ok = mbar_wait_bounded(&raw_bar[rs], (i / RAWS) & 1, prm.wait_ns);
       ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
       if (!ok) {
         if (lane == 0) {
@@ -365,17 +364,29 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
         }
         break;
       }
+      // The weight tile goes out as soon as its stage is free; the
+      // activation slab it is used with is converted while it streams in.
       uint8_t* stage = smem + st * SL::kBytes;
       if (lane == 0) {
         const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, ps));
         mbar_arrive_expect_tx(&full_bar[st], tbytes);
         bulk_copy_g2s(stage, prm.packed + tile_offset(g, ps, pb), tbytes, &full_bar[st]);
       }
+      issued = i + 1;
+      ok = mbar_wait_bounded(&raw_bar[rs], (i / RAWS) & 1, prm.wait_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
+      if (!ok) {
+        if (lane == 0) {
+          atomicOr(prm.err, kDevErrTimeout);
+          *abort_flag = 1;
+        }
+        mbar_arrive(&full_bar[st]);      // let the stage's phase complete once the copy lands
+        break;
+      }
       XSlice<MP, MIXED> xs;
       read_x_slice<MP, MIXED>(xs, raw_ring + rs * SL::kRawBytes, prm, ps, lane);
       store_x_slice<MP, MIXED>(xs, stage, prm, lane);
       mbar_arrive(&full_bar[st]);
-      issued = i + 1;
       ps = next_slab(ps);
       if (ps == 0) ++pb;
       __syncwarp();                      // every lane has read raw slot rs
@@ -621,8 +632,22 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
             for (int e = lane; e < kRowsPerCounter * prm.M; e += 32) {
               const int n = b * kTileRows + warp * kRowsPerCounter + (e % kRowsPerCounter);
               const int m = e / kRowsPerCounter;
+              // the pieces' partials, eight loads in flight at a time, added in
+              // slab order
               float tot = 0.0f;
-              for (int c2 = c_first; c2 <= c_last; ++c2) {
+              int c2 = c_first;
+              for (; c2 + 7 <= c_last; c2 += 8) {
+                float v8[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                  const long long tc = (long long)(c2 + t) * prm.tiles / G;
+                  const int sa = (int)((tc > ub ? tc : ub) - ub);
+                  v8[t] = __ldcg(prm.partials + ((size_t)sa * MP + m) * g.Npad + n);
+                }
+#pragma unroll
+                for (int t = 0; t < 8; ++t) tot += v8[t];
+              }
+              for (; c2 <= c_last; ++c2) {
                 const long long tc = (long long)c2 * prm.tiles / G;
                 const int sa = (int)((tc > ub ? tc : ub) - ub);
                 tot += __ldcg(prm.partials + ((size_t)sa * MP + m) * g.Npad + n);
