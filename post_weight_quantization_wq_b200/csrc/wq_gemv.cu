@@ -293,10 +293,26 @@ __device__ __forceinline__ void store_x_slice(const XSlice<MP, MIXED>& xs, uint8
   }
 }
 
-template <int MP, int JQ, int STAGES, int RAWS, int MINB, bool MIXED>
-__global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvParams prm) {
+// Bytes of shared memory one (virtual) CTA of the GEMV uses, rounded to 128.
+template <int MP, int STAGES, int RAWS, bool MIXED>
+__host__ __device__ constexpr size_t gemv_team_smem() {
+  return ((size_t)STAGES * StageLayout<MP, MIXED>::kBytes +
+          (size_t)RAWS * StageLayout<MP, MIXED>::kRawBytes + (2 * STAGES + RAWS) * 8 + 16 + 127) /
+         128 * 128;
+}
+
+// One CTA per SM runs VC independent teams ("virtual CTAs"), each a producer
+// warp and kConsumerWarps consumer warps with its own shared memory and its
+// own contiguous run of tiles.  The team of a warp is its warp index mod VC,
+// so every team gets warps of every age: CTAs sharing an SM are not scheduled
+// evenly (the older CTA's warps win the issue slots), teams inside one CTA
+// are, and the SM's work then finishes at the same time.
+template <int MP, int JQ, int STAGES, int RAWS, int VC, bool MIXED>
+__global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvParams prm) {
   using SL = StageLayout<MP, MIXED>;
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem_all[];
+  const int team = (threadIdx.x >> 5) % VC;
+  uint8_t* smem = smem_all + team * gemv_team_smem<MP, STAGES, RAWS, MIXED>();
   const Geom g = prm.g;
   uint8_t* raw_ring = smem + STAGES * SL::kBytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(raw_ring + RAWS * SL::kRawBytes);
@@ -304,14 +320,16 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
   uint64_t* raw_bar = empty_bar + STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(raw_bar + RAWS);
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = (threadIdx.x >> 5) / VC;     // warp index within the team
   const int lane = threadIdx.x & 31;
-  const int G = gridDim.x;
-  const long long t0 = (long long)blockIdx.x * prm.tiles / G;
-  const long long t1 = (long long)(blockIdx.x + 1) * prm.tiles / G;
+  const int ltid = warp * 32 + lane;           // thread index within the team
+  const int G = gridDim.x * VC;                // teams of the grid
+  const int vb = blockIdx.x * VC + team;       // this team's index
+  const long long t0 = (long long)vb * prm.tiles / G;
+  const long long t1 = (long long)(vb + 1) * prm.tiles / G;
   const int ntiles = (int)(t1 - t0);
 
-  if (threadIdx.x == 0) {
+  if (ltid == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full_bar[i], 1 + 32);           // producer's expect_tx + its 32 lanes
       mbar_init(&empty_bar[i], kConsumerWarps);
@@ -322,7 +340,7 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
   }
   // Rows of x beyond M are never written: zero every stage's activation area once.
   for (int st = 0; st < STAGES; ++st)
-    for (int i = threadIdx.x; i < (SL::kBytes - SL::kX) / 16; i += blockDim.x)
+    for (int i = ltid; i < (SL::kBytes - SL::kX) / 16; i += kGemvThreads)
       reinterpret_cast<uint4*>(smem + st * SL::kBytes + SL::kX)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
 
@@ -672,15 +690,15 @@ __global__ void __launch_bounds__(kGemvThreads, MINB) gemv_w4a16_kernel(GemvPara
 struct GemvConfig {
   const void* fn;
   size_t smem;
+  int teams;               // virtual CTAs per CTA
 };
 
-template <int MP, int JQ, int STAGES, int RAWS, int MINB, bool MIXED>
+template <int MP, int JQ, int STAGES, int RAWS, int VC, bool MIXED>
 static GemvConfig gemv_config() {
-  using SL = StageLayout<MP, MIXED>;
   GemvConfig c;
-  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, RAWS, MINB, MIXED>);
-  c.smem = (size_t)STAGES * SL::kBytes + (size_t)RAWS * SL::kRawBytes +
-           (2 * STAGES + RAWS) * sizeof(uint64_t) + 16;
+  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, RAWS, VC, MIXED>);
+  c.smem = VC * gemv_team_smem<MP, STAGES, RAWS, MIXED>();
+  c.teams = VC;
   return c;
 }
 
@@ -729,12 +747,15 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
 
   const GemvConfig c = pick_gemv(M, inv_s != nullptr);
   int per_sm = 0;
-  cudaError_t e = kernel_setup(c.fn, c.smem, kGemvThreads, &per_sm);
+  cudaError_t e = kernel_setup(c.fn, c.smem, kGemvThreads * c.teams, &per_sm);
   if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
   long long grid = (long long)num_sms * per_sm;
-  if (grid > prm.tiles) grid = prm.tiles;
+  const long long need = (prm.tiles + c.teams - 1) / c.teams;
+  if (grid > need) grid = need;
   void* args[] = {&prm};
-  return cudaLaunchKernel(c.fn, dim3((unsigned)grid), dim3(kGemvThreads), args, c.smem, stream);
+  return cudaLaunchKernel(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem,
+                          stream);
 }
 
 }  // namespace wq
