@@ -278,6 +278,7 @@ def run_ours(a, rank: int, world: int, local_rank: int):
         del copies, qw
         torch.cuda.empty_cache()
         extras["gemm"] = time_gemm(dev, stream)
+        extras["layer_awq"] = time_layer_awq(dev, stream)
     line.update(extras)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(W, x, N, K, sym)
@@ -444,6 +445,76 @@ def time_gemm(dev, stream):
         torch.cuda.empty_cache()
     if abi.wq_last_device_status(stream) != 0:
         raise RuntimeError("device error in the GEMM leg")
+    return out
+
+
+def time_layer_awq(dev, stream):
+    """The AWQ workload: the seven linears of a Llama-70B GQA decoder layer
+    (q, k, v, o, gate, up, down; 455 MB packed, more than L2) quantized with
+    the AWQ scale folded in, run in order through wq_gemv_w4a16 with the
+    activation factor 1/s, as one CUDA graph; M = 1 and 4."""
+    import numpy as np
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    from post_weight_quantization_wq_b200 import _binding as abi
+    from post_weight_quantization_wq_b200 import inputs
+    cid = 5
+    wl = inputs.WORKLOADS[cid]
+    lins = []
+    for li, lin in enumerate(wl.linears):
+        W = inputs.workload_weight(cid, li)
+        s_awq = inputs.workload_awq_scale(cid, li)
+        Wt = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+        del W
+        s_t = torch.from_numpy(s_awq).to(dev)
+        qw = wq.quantize(Wt, awq_scale=s_t, symmetric=wl.sym, stream=stream)
+        torch.cuda.synchronize(dev)
+        del Wt
+        inv = (1.0 / s_t.double()).float()
+        lins.append((lin, qw, inv))
+    out = {}
+    for M in wl.Ms:
+        runs = []
+        nbytes = 0
+        for li, (lin, qw, inv) in enumerate(lins):
+            x = inputs.workload_activations(cid, li, M)
+            xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((M, lin.N), dtype=torch.float32, device=dev)
+            wsb = abi.wq_workspace_bytes(M, lin.N, lin.K)
+            ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)
+            runs.append((lin, qw, inv, xt, y, ws, wsb))
+            nbytes += algorithmic_bytes(M, lin.N, lin.K, wl.sym)
+
+        def layer(s):
+            for lin, qw, inv, xt, y, ws, wsb in runs:
+                st = abi.wq_gemv_w4a16(xt, inv, qw.packed, M, lin.N, lin.K, 128, wl.sym, 1, y, ws,
+                                       wsb, s)
+                assert st == 0
+
+        with torch.cuda.stream(stream):
+            layer(stream)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        reps = 20
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                layer(stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g.replay()
+            e0.record(stream)
+            for _ in range(10):
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (10 * reps)
+        out[f"m{M}"] = {"us_per_layer": round(us, 2), "bytes": nbytes,
+                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "launches": 7}
+    if abi.wq_last_device_status(stream) != 0:
+        raise RuntimeError("device error in the AWQ layer leg")
+    del lins
+    torch.cuda.empty_cache()
     return out
 
 

@@ -6,7 +6,8 @@ PyTorch and calls the ABI through :mod:`._binding`.  There is no CPU path:
 every function here raises if the library or a GPU is missing.
 
     qw = quantize(W)                 # wq_quantize_rtn + wq_pack_layout
-    y = linear(x, qw)                # wq_gemv_w4a16 (M <= 8) / wq_gemm_w4a16 (M >= 16)
+    y = linear(x, qw)                # wq_gemv_w4a16 (M <= 2, or with the AWQ factor) /
+                                     # wq_gemm_w4a16 (tensor cores, M >= 3)
 """
 from __future__ import annotations
 
