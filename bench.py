@@ -43,8 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": "ae6901fba59f04aba69bd6ccd46a6aeffdea60649770259e8285ca2b67d029bd",
-               "bytes_per_launch": 124904192 + 4314112}
+NCU_TRAFFIC = {"sources_sha256": "742a2f5e32bcaeb452ac6e0c8393cdaa388df67f5a9e5b9fc9a962acdeddfb82",
+               "bytes_per_launch": 124905984 + 3631616}
 
 
 def _args():
