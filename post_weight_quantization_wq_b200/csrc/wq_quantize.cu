@@ -31,53 +31,69 @@ struct QuantParams {
 };
 
 struct GroupResult {
-  uint32_t word;
+  uint32_t word0, word1;   // this lane's two packed words
   uint16_t s16, z16;
   bool bad;
 };
 
-// One half-warp (16 lanes) quantizes one group; lane `hl` holds elements
-// 8*hl .. 8*hl+7 of the group, so it produces exactly one packed word.
-__device__ __forceinline__ GroupResult quantize_group(const uint4 raw, const float* awq_k,
-                                                      unsigned mask, int sym) {
-  float w[8];
-  const uint32_t r32[4] = {raw.x, raw.y, raw.z, raw.w};
+// Round-to-nearest-even of w / sf for one element, given r = RN(1 / sf).
+// t = RN(w * r) is within |t| * 2^-23 (plus rounding) of the exact quotient,
+// so when t is farther than |t| * 2^-20 + 2^-24 from the nearest half-integer
+// the correctly rounded quotient RN(w / sf) rounds to the same integer as t;
+// otherwise (rare: near a tie, or |t| >= 2^20) the IEEE division decides.
+__device__ __forceinline__ float round_quotient(float w, float sf, float r) {
+  const float t = __fmul_rn(w, r);
+  const float fl = floorf(t);
+  const float d = fabsf(__fsub_rn(__fsub_rn(t, fl), 0.5f));
+  if (d > __fmaf_rn(fabsf(t), 0x1p-20f, 0x1p-24f)) return rintf(t);
+  return rintf(__fdiv_rn(w, sf));
+}
+
+// Eight lanes (a quarter warp, `mask`) quantize one group; lane ql holds
+// elements 16*ql .. 16*ql+15 of the group, so it produces two packed words.
+__device__ __forceinline__ GroupResult quantize_group(const uint4 raw0, const uint4 raw1,
+                                                      const float* awq_k, unsigned mask,
+                                                      int sym) {
+  float w[16];
+  const uint32_t r32[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 8; ++i) {
     w[2 * i] = __uint_as_float(r32[i] << 16);
     w[2 * i + 1] = __uint_as_float(r32[i] & 0xFFFF0000u);
   }
   if (awq_k) {
-    const float4 a0 = __ldg(reinterpret_cast<const float4*>(awq_k));
-    const float4 a1 = __ldg(reinterpret_cast<const float4*>(awq_k) + 1);
-    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(w[i], a[i]);   // W' = W diag(s)
+    for (int v = 0; v < 4; ++v) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(awq_k) + v);
+      w[4 * v + 0] = __fmul_rn(w[4 * v + 0], a.x);   // W' = W diag(s)
+      w[4 * v + 1] = __fmul_rn(w[4 * v + 1], a.y);
+      w[4 * v + 2] = __fmul_rn(w[4 * v + 2], a.z);
+      w[4 * v + 3] = __fmul_rn(w[4 * v + 3], a.w);
+    }
   }
   bool bad = false;
-  float amax = 0.0f, mn = w[0], mx = w[0];
+  float mn = w[0], mx = w[0];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 16; ++i) {
     bad |= !isfinite(w[i]);
-    amax = fmaxf(amax, fabsf(w[i]));
     mn = fminf(mn, w[i]);
     mx = fmaxf(mx, w[i]);
   }
   bad = __any_sync(mask, bad);
 #pragma unroll
-  for (int o = 8; o >= 1; o >>= 1) {
-    amax = fmaxf(amax, __shfl_xor_sync(mask, amax, o));
+  for (int o = 4; o >= 1; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(mask, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(mask, mx, o));
   }
 
   GroupResult res;
-  res.word = 0;
+  res.word0 = res.word1 = 0;
   res.s16 = 0;
   res.z16 = 0;
   float sf = 1.0f, zf = 0.0f;
   if (!bad) {
-    float range = sym ? amax : __fsub_rn(mx, mn);
+    // symmetric range max|w| = max(-min, max), exactly
+    float range = sym ? fmaxf(-mn, mx) : __fsub_rn(mx, mn);
     if (range < 1e-8f) range = 1e-8f;
     const float s32 = __fdiv_rn(range, sym ? 7.0f : 15.0f);
     uint16_t hs = __half_as_ushort(__float2half_rn(s32));
@@ -99,48 +115,53 @@ __device__ __forceinline__ GroupResult quantize_group(const uint4 raw, const flo
     res.z16 = 0x7E00;
     return res;
   }
+  const float r = __frcp_rn(sf);
   const float lo = sym ? -7.0f : 0.0f, hi = sym ? 7.0f : 15.0f;
-  uint32_t word = 0;
+  uint32_t word[2] = {0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float t = __fadd_rn(rintf(__fdiv_rn(w[i], sf)), zf);
+  for (int i = 0; i < 16; ++i) {
+    float t = __fadd_rn(round_quotient(w[i], sf, r), zf);
     t = fminf(fmaxf(t, lo), hi);
     const int code = static_cast<int>(t) + (sym ? 8 : 0);
-    word |= static_cast<uint32_t>(code & 0xF) << (4 * i);
+    word[i >> 3] |= static_cast<uint32_t>(code & 0xF) << (4 * (i & 7));
   }
-  res.word = word;
+  res.word0 = word[0];
+  res.word1 = word[1];
   res.bad = false;
   return res;
 }
 
 __global__ void __launch_bounds__(256) quantize_rtn_kernel(QuantParams p) {
   const int lane = threadIdx.x & 31;
-  const int hl = lane & 15;
-  const unsigned mask = (lane < 16) ? 0x0000FFFFu : 0xFFFF0000u;
-  const long long nhalf = (long long)gridDim.x * (blockDim.x / 16);
-  long long gid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 16;
+  const int ql = lane & 7;
+  const unsigned mask = 0xFFu << (lane & 24);      // this quarter warp
+  const long long nq = (long long)gridDim.x * (blockDim.x / 8);
+  long long gid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 8;
 
-  // Two groups per iteration so each lane keeps two 16-byte loads in flight.
-  for (; gid < p.groups; gid += 2 * nhalf) {
-    const long long gid2 = gid + nhalf;
+  // Two groups per iteration so each lane keeps four 16-byte loads in flight.
+  for (; gid < p.groups; gid += 2 * nq) {
+    const long long gid2 = gid + nq;
     const bool has2 = gid2 < p.groups;
-    const uint4 raw1 = __ldcs(p.W + gid * 16 + hl);
-    uint4 raw2 = make_uint4(0, 0, 0, 0);
-    if (has2) raw2 = __ldcs(p.W + gid2 * 16 + hl);
-
-    const float* a1 = p.awq ? p.awq + (gid % p.NG) * kGroup + 8 * hl : nullptr;
-    GroupResult r1 = quantize_group(raw1, a1, mask, p.sym);
-    p.qweight[gid * 16 + hl] = r1.word;
-    if (hl == 0) {
+    const uint4 a0 = __ldcs(p.W + gid * 16 + 2 * ql);
+    const uint4 a1 = __ldcs(p.W + gid * 16 + 2 * ql + 1);
+    uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+    if (has2) {
+      b0 = __ldcs(p.W + gid2 * 16 + 2 * ql);
+      b1 = __ldcs(p.W + gid2 * 16 + 2 * ql + 1);
+    }
+    const float* s1 = p.awq ? p.awq + (gid % p.NG) * kGroup + 16 * ql : nullptr;
+    const GroupResult r1 = quantize_group(a0, a1, s1, mask, p.sym);
+    reinterpret_cast<uint2*>(p.qweight)[gid * 8 + ql] = make_uint2(r1.word0, r1.word1);
+    if (ql == 0) {
       p.scales[gid] = r1.s16;
       if (!p.sym) p.zeros[gid] = r1.z16;
       if (r1.bad && p.d_status) atomicAdd(p.d_status, 1);
     }
     if (has2) {
-      const float* a2 = p.awq ? p.awq + (gid2 % p.NG) * kGroup + 8 * hl : nullptr;
-      GroupResult r2 = quantize_group(raw2, a2, mask, p.sym);
-      p.qweight[gid2 * 16 + hl] = r2.word;
-      if (hl == 0) {
+      const float* s2 = p.awq ? p.awq + (gid2 % p.NG) * kGroup + 16 * ql : nullptr;
+      const GroupResult r2 = quantize_group(b0, b1, s2, mask, p.sym);
+      reinterpret_cast<uint2*>(p.qweight)[gid2 * 8 + ql] = make_uint2(r2.word0, r2.word1);
+      if (ql == 0) {
         p.scales[gid2] = r2.s16;
         if (!p.sym) p.zeros[gid2] = r2.z16;
         if (r2.bad && p.d_status) atomicAdd(p.d_status, 1);
@@ -229,8 +250,8 @@ cudaError_t launch_quantize(const void* W, const float* awq, int N, int K, int s
     cudaError_t e = cudaMemsetAsync(d_status, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;
   }
-  const long long halves_needed = (p.groups + 1) / 2;
-  long long blocks = (halves_needed + 15) / 16;
+  const long long quarters_needed = (p.groups + 1) / 2;   // two groups per quarter warp
+  long long blocks = (quarters_needed + 31) / 32;
   const long long cap = (long long)num_sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
