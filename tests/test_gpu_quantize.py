@@ -65,3 +65,38 @@ def test_quantize_awq_overflow_is_nonfinite():
 def test_quantize_outlier_weights_config2_shape():
     W = inputs.weights(512, 4096, 0.02, seed=2000, outlier_frac=0.001)
     quantize_and_check(W, None, True)
+
+
+def _near_tie_inputs(sym):
+    """W = 1.0 everywhere and an AWQ scale that places each w' = fp32(1 * s_k)
+    exactly where its quotient by the group's fp16 scale lies just beside a
+    half-integer (by 0 to 1e-4 relative, both sides) or on it: the quantizer
+    must round every one exactly as an IEEE division would."""
+    r = np.random.default_rng(12)
+    K, N = 128 * 8, 4
+    s_awq = np.empty(K, np.float32)
+    for g in range(K // 128):
+        amax = np.float32(r.uniform(0.3, 3.0))
+        if sym:
+            s16 = np.float16(amax / np.float32(7.0))
+            lo, hi = -7, 6
+        else:
+            s16 = np.float16((amax - (-amax)) / np.float32(15.0))
+            lo, hi = -8, 6
+        vals = [amax, -amax]
+        rel = [0.0, 1e-9, 1e-8, 1e-7, 5e-7, 1e-6, 3e-6, 1e-5, 1e-4]
+        while len(vals) < 128:
+            m = r.integers(lo, hi + 1)
+            d = rel[r.integers(len(rel))] * (1 if r.random() < 0.5 else -1)
+            v = np.float32(np.float64(s16) * (m + 0.5) * (1.0 + d))
+            if abs(v) < amax:
+                vals.append(v)
+        s_awq[g * 128:(g + 1) * 128] = np.array(vals, np.float32)
+    W = inputs.to_bf16_bits(np.ones((N, K), np.float32))
+    return W, s_awq
+
+
+@pytest.mark.parametrize("sym", [True, False])
+def test_quantize_near_ties(sym):
+    W, s_awq = _near_tie_inputs(sym)
+    quantize_and_check(W, s_awq, sym)
