@@ -143,6 +143,21 @@ wq_status check_linear(const void* x, const float* inv_s, const void* packed, in
 }  // namespace
 
 namespace wq {
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, void** args, size_t smem,
+                       cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 // Error-word address, SM count and wait limit of the current device (set up
 // on first use), for entry points defined in other files of the library.
 cudaError_t device_info(int** err, int* num_sms, unsigned long long* wait_ns) {

@@ -157,6 +157,23 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Programmatic dependent launch (sm_90+): wait until the previous kernel of
+// the stream has completed and its memory is visible (a no-op when this grid
+// was not launched as a programmatic dependent), and allow the next kernel of
+// the stream to start early.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Host: launch `fn` so that it may start while the previous kernel of the
+// stream finishes (it must call griddep_wait before touching what that
+// kernel writes).
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, void** args, size_t smem,
+                       cudaStream_t stream);
+
 // Host: once per (device, kernel, dynamic smem size), raise the kernel's
 // dynamic shared-memory limit and query how many CTAs fit on one SM.  Later
 // calls only read the cache, so launches issued during stream capture make no

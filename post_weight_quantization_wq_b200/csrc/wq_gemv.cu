@@ -343,6 +343,10 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
     for (int i = ltid; i < (SL::kBytes - SL::kX) / 16; i += kGemvThreads)
       reinterpret_cast<uint4*>(smem + st * SL::kBytes + SL::kX)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
+  // Programmatic dependent launch: the next kernel in the stream may start
+  // as soon as SMs free up (it waits for this grid before it touches
+  // anything this grid writes).
+  griddep_launch_dependents();
 
   if (warp == kConsumerWarps) {
     // ---------------------------------------------------------------- producer
@@ -362,6 +366,22 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
                       &raw_bar[slot]);
       if (ib) bulk_copy_g2s(dst + SL::kRawInv, prm.inv_s + slab * kSlabK, ib, &raw_bar[slot]);
     };
+    // The first STAGES weight tiles do not depend on the previous kernel in
+    // the stream (no kernel of this library writes weights): they go out
+    // before the wait for it, so they stream in while that kernel finishes.
+    const int early = ntiles < STAGES ? ntiles : STAGES;
+    if (lane == 0) {
+      int eb = pb, es = ps;
+      for (int k = 0; k < early; ++k) {
+        const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, es));
+        mbar_arrive_expect_tx(&full_bar[k], tbytes);
+        bulk_copy_g2s(smem + k * SL::kBytes, prm.packed + tile_offset(g, es, eb), tbytes,
+                      &full_bar[k]);
+        es = next_slab(es);
+        if (es == 0) ++eb;
+      }
+    }
+    griddep_wait();                      // x, y and the workspace may belong to it
     if (lane == 0)
       for (int r = 0; r < RAWS && r < ntiles; ++r) {
         issue_raw(r, pf);
@@ -385,7 +405,7 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
       // The weight tile goes out as soon as its stage is free; the
       // activation slab it is used with is converted while it streams in.
       uint8_t* stage = smem + st * SL::kBytes;
-      if (lane == 0) {
+      if (lane == 0 && i >= early) {
         const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, ps));
         mbar_arrive_expect_tx(&full_bar[st], tbytes);
         bulk_copy_g2s(stage, prm.packed + tile_offset(g, ps, pb), tbytes, &full_bar[st]);
@@ -432,6 +452,7 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
   }
 
   // ------------------------------------------------------------------ consumers
+  griddep_wait();                      // y and the workspace may belong to the previous kernel
   const int rq = lane >> 3;         // row of the quad handled by this lane group
   const int p = lane & 7;           // 64-input chunk of the slab
   constexpr int V = JQ * MP;
@@ -754,8 +775,8 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   const long long need = (prm.tiles + c.teams - 1) / c.teams;
   if (grid > need) grid = need;
   void* args[] = {&prm};
-  return cudaLaunchKernel(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem,
-                          stream);
+  return launch_pdl(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem,
+                    stream);
 }
 
 }  // namespace wq
