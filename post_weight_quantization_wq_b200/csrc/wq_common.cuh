@@ -100,6 +100,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same condition.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // As mbar_try_wait, but a thread whose phase has not completed is suspended
 // (it issues nothing) until the phase completes or about `hint_ns`
 // nanoseconds have passed.
@@ -127,11 +139,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // the issue slots to the working ones.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns) {
+  if (limit_ns < 20000u) {
+    // a short limit (the timeout test hook): poll with the non-blocking
+    // test_wait (try_wait may itself wait for a while), so the limit holds
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  const uint32_t hint = limit_ns < 20000u ? (uint32_t)limit_ns + 1u : 20000u;
   while (true) {
-    if (mbar_try_wait_suspend(bar, parity, hint)) return true;
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
