@@ -43,8 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": "742a2f5e32bcaeb452ac6e0c8393cdaa388df67f5a9e5b9fc9a962acdeddfb82",
-               "bytes_per_launch": 124905984 + 3631616}
+NCU_TRAFFIC = {"sources_sha256": "241a2691d2f78add74c29ff11e6561ba6cbc80dc9e670a8d6ac018ffb8b94e27",
+               "bytes_per_launch": 124908544 + 3814400}
 
 
 def _args():
