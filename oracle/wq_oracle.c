@@ -24,7 +24,7 @@
  *           (Y = X W^T, W: [out_features, in_features], groups along
  *           in_features), section dtype、storage dtype、compute dtype.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - the integer codes are computed with the fp16-rounded scale s16 (the
  *     stored one) and, for the asymmetric form, with the fp16-stored zero z16,
  *     so the stored metadata reproduce x_hat exactly;
