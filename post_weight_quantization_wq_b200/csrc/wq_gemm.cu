@@ -1,13 +1,14 @@
-// wq_gemm.cu -- W4A16 skinny GEMM for M = 16..64 activation rows on the 5th-
+// wq_gemm.cu -- W4A16 skinny GEMM for M = 1..64 activation rows on the 5th-
 // generation tensor cores (tcgen05, sm_100a):
 //
 //   y[m][n] = sum_g s16[n][g] * sum_{k in g} x[m][k] * (q[n][k] - z[n][g])
 //
-// At 16..64 rows the product is a dense contraction, so the dequantized
-// weights go through the tensor cores ("3.6 量化(Quantization)", section
-// 仅权重 vs 权重 + 激活: the 4-bit weights are dequantized to 16-bit inside the
-// matmul kernel; "大模型量化全景解析", section dtype、storage dtype、compute
-// dtype: 16-bit compute, higher-precision accumulation).
+// With several rows of x the product is a dense contraction, so the
+// dequantized weights go through the tensor cores ("3.6 量化(Quantization)",
+// section 仅权重 vs 权重 + 激活: the 4-bit weights are dequantized to 16-bit
+// inside the matmul kernel; "大模型量化全景解析", section dtype、storage dtype、
+// compute dtype: 16-bit compute, higher-precision accumulation).  x is
+// zero-padded by its tensor map to Mpad = 16, 32, 48 or 64 rows.
 //
 // Per group of 128 inputs, the weight tile A (128 output rows x 128 inputs)
 // holds the bf16 integers 128 + q (exact), x arrives as the bf16 tile B
@@ -18,16 +19,19 @@
 // never enter the bf16 operands, so any stored z is handled exactly.
 //
 // Data flow of one CTA (persistent, one per SM, contiguous run of layout
-// tiles u = b * NS + s like the GEMV), per group of 128 inputs:
+// tiles u = b * NS + s like the GEMV).  The roles hand work to each other in
+// stages of two consecutive groups of the CTA's group sequence (one mbarrier
+// handoff per 256 inputs); per group:
 //   codes   2-D TMA load of the group's 128 rows x 64 B of codes out of the
 //           packed tile (SWIZZLE_64B, so that a warp reading 32 rows at one
-//           column offset touches every bank once) into a 12..16-slot ring;
+//           column offset touches every bank once) into a ring of 6..8
+//           stages; the tile's metadata by one bulk copy per tile;
 //   A       the dequantizing warps turn each row's 16 code words into 64
 //           bf16 pairs and store them into tensor memory (tcgen05.st): the
 //           A operand never passes through shared memory;
 //   x       2-D TMA loads of the bf16 activation tile (SWIZZLE_128B, rows >= M
-//           zero-filled) into a 4-slot ring, and a bulk copy of the group's
-//           precomputed sum(x) row into an 8-slot ring;
+//           zero-filled), and a bulk copy of the group's precomputed sum(x)
+//           row;
 //   MMA     one lane issues 8 tcgen05.mma (M=128, N=Mpad, K=16, A in tensor
 //           memory, B in shared memory) into one of 4 accumulators;
 //   fold    one thread per output row reads its accumulator row (tcgen05.ld)
@@ -37,9 +41,9 @@
 // Warps: 0 code producer, 1 tensor-memory owner and MMA issuer, 2
 // activation producer, 4-11 dequantize (inputs 0-63 and 64-127 of each
 // group, one warp per lane quadrant), 12-19 fold (columns 0..Mpad/2-1 and
-// Mpad/2..Mpad-1 of the accumulator, one warp per lane quadrant).  Every wait is bounded; on timeout the kernel records
-// the device error word and winds down (waiting, bounded, for its copies and
-// MMAs in flight).
+// Mpad/2..Mpad-1 of the accumulator, one warp per lane quadrant).  Every
+// wait is bounded; on timeout the kernel records the device error word and
+// winds down (waiting, bounded, for its copies and MMAs in flight).
 #include <cuda.h>
 #include <cstring>
 #include <cudaTypedefs.h>
