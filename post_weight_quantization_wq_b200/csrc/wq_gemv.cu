@@ -9,16 +9,19 @@
 // section dtype、storage dtype、compute dtype).
 //
 // Design (B200, sm_100a):
-//   * persistent grid; CTA c owns the contiguous run [t0, t1) of the tile
-//     sequence u = b * NS + s (row tile b of 128 output rows, K-slab s of 512
-//     inputs), so it walks the slabs of one row tile after another and keeps
-//     each row's running sum in registers;
-//   * a producer warp streams every tile (32 KB of nibbles + its fp16
-//     metadata, contiguous in memory) into a ring of shared-memory stages with
-//     one 1-D bulk async copy (cp.async.bulk) completing on an mbarrier, and
-//     prepares the tile's activation slab once for the whole CTA: bf16 x plus
-//     fp32 sums of x per 64 inputs (mixed path), or fp32 x * (1/s) (packed
-//     path); eight consumer warps compute;
+//   * persistent grid of one CTA per SM holding 1..3 teams (a producer warp
+//     and eight consumer warps each, with their own shared memory); team t
+//     owns the contiguous run [t0, t1) of the tile sequence u = b * NS + s
+//     (row tile b of 128 output rows, K-slab s of 512 inputs), so it walks
+//     the slabs of one row tile after another and keeps each row's running
+//     sum in registers;
+//   * the producer streams every tile (32 KB of nibbles + its fp16 metadata,
+//     contiguous in memory) into a ring of shared-memory stages with one 1-D
+//     bulk async copy (cp.async.bulk) completing on an mbarrier, and prepares
+//     the tile's activation slab once for the team: bf16 x plus fp32 sums of
+//     x per 64 inputs (mixed path), or fp32 x * (1/s) (packed path);
+//   * programmatic dependent launch: the first weight tiles are requested
+//     before the kernel waits for the previous kernel of the stream;
 //   * dequantization in registers, two codes per LOP3 (no conversion
 //     instruction): mixed path (no activation scale, M <= 4): masked nibble
 //     pairs OR-ed into fp16 exponent patterns are 1024 + q or 64 + q exactly
@@ -32,11 +35,11 @@
 //   * 8 lanes share a row of a tile, lane p covering inputs 64p..64p+63 of
 //     the slab; their partial sums of several rows are combined with a
 //     transposing shuffle reduction;
-//   * a row tile whose slabs are split between CTAs (only at the ends of a
-//     CTA's run) is finished through the workspace: each piece writes its
+//   * a row tile whose slabs are split between teams (only at the ends of a
+//     team's run) is finished through the workspace: each piece writes its
 //     fp32 partial, and the last piece to arrive (an atomic counter per 16
 //     rows) adds the pieces in slab order and resets the counter, so y does
-//     not depend on the order the GPU runs the CTAs in;
+//     not depend on the order the GPU runs the teams in;
 //   * every wait is bounded (globaltimer): on timeout the kernel records the
 //     device error word, stops issuing copies, waits (bounded) for its copies
 //     in flight and returns.
