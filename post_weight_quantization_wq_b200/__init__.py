@@ -25,6 +25,24 @@ def _check(status: int, where: str) -> None:
         raise WqError(status, where)
 
 
+def _require(t, name: str, dtype, shape=None, device=None):
+    """The C ABI takes raw device pointers: refuse anything it would misread
+    (host memory, another dtype, a strided view, a wrong shape or GPU)."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor (got {t.device})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
 @dataclass
 class QuantizedWeight:
     """A quantized weight: canonical buffers plus the kernel-layout copy."""
@@ -43,8 +61,13 @@ def quantize(W, awq_scale=None, symmetric: bool = False, stream=None,
     """Quantize a bf16 CUDA tensor W [N][K] (optionally with the AWQ scale
     folded in) and lay it out for the linear kernels."""
     import torch
+    if getattr(W, "dim", lambda: 0)() != 2:
+        raise ValueError("W: expected a 2-D tensor [N][K]")
     N, K = W.shape
+    _require(W, "W", torch.bfloat16)
     dev = W.device
+    if awq_scale is not None:
+        _require(awq_scale, "awq_scale", torch.float32, (K,), dev)
     qweight = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
     scales = torch.empty((N, K // GROUP), dtype=torch.float16, device=dev)
     zeros = None if symmetric else torch.empty((N, K // GROUP), dtype=torch.float16, device=dev)
@@ -62,15 +85,16 @@ def quantize(W, awq_scale=None, symmetric: bool = False, stream=None,
 _workspaces = {}
 
 
-def workspace_for(M: int, N: int, K: int, device, path: str = "gemv"):
+def workspace_for(M: int, N: int, K: int, device, path: str = "gemv", stream=None):
     """A zero-filled workspace large enough for (M, N, K) on the given path,
-    cached per device (it only grows)."""
+    cached per (device, stream) -- calls that share a workspace must not run
+    concurrently -- and only ever grown."""
     import torch
     need = abi.wq_gemm_workspace_bytes(M, N, K) if path == "gemm" else \
         abi.wq_workspace_bytes(M, N, K)
     if need == 0:
         return None, 0
-    key = (str(device),)
+    key = (str(device), abi._stream(stream))
     ws = _workspaces.get(key)
     if ws is None or ws.numel() < need:
         ws = torch.zeros(need, dtype=torch.uint8, device=device)
@@ -87,8 +111,16 @@ def linear(x, qw: QuantizedWeight, inv_act_scale=None, out=None, workspace=None,
     path: None (choose by M), "gemv" (wq_gemv_w4a16, M <= 8) or "gemm"
     (wq_gemm_w4a16, tensor cores, no AWQ factor)."""
     import torch
+    if getattr(x, "dim", lambda: 0)() != 2:
+        raise ValueError("x: expected a 2-D tensor [M][K]")
     M, K = x.shape
-    assert K == qw.K
+    _require(x, "x", torch.bfloat16, (M, qw.K), qw.packed.device)
+    if inv_act_scale is not None:
+        _require(inv_act_scale, "inv_act_scale", torch.float32, (K,), x.device)
+    if out is not None:
+        _require(out, "out", torch.float32, (M, qw.N), x.device)
+    if workspace is not None:
+        _require(workspace, "workspace", torch.uint8, None, x.device)
     y = out if out is not None else torch.empty((M, qw.N), dtype=torch.float32, device=x.device)
     # CUDA-core GEMV up to 2 rows (HBM-bound) and for the AWQ fold (its
     # scaled activations are not exact in a bf16 tensor-core operand);
@@ -96,7 +128,7 @@ def linear(x, qw: QuantizedWeight, inv_act_scale=None, out=None, workspace=None,
     if path is None:
         path = "gemv" if (M <= GEMV_MAX_ROWS or inv_act_scale is not None) else "gemm"
     if workspace is None:
-        ws, ws_bytes = workspace_for(M, qw.N, K, x.device, path)
+        ws, ws_bytes = workspace_for(M, qw.N, K, x.device, path, stream)
     else:
         ws, ws_bytes = workspace, workspace.numel()
     fn = abi.wq_gemv_w4a16 if path == "gemv" else abi.wq_gemm_w4a16
