@@ -18,20 +18,22 @@
 //   * the producer streams every tile (32 KB of nibbles + its fp16 metadata,
 //     contiguous in memory) into a ring of shared-memory stages with one 1-D
 //     bulk async copy (cp.async.bulk) completing on an mbarrier, and prepares
-//     the tile's activation slab once for the team: bf16 x plus fp32 sums of
-//     x per 64 inputs (mixed path), or fp32 x * (1/s) (packed path);
+//     the tile's activation slab once for the team: 16-bit fixed-point x
+//     (split into high and low bytes) plus the sum of x per 64 inputs
+//     (integer path), or fp32 x * (1/s) (packed path);
 //   * programmatic dependent launch: the first weight tiles are requested
 //     before the kernel waits for the previous kernel of the stream;
-//   * dequantization in registers, two codes per LOP3 (no conversion
-//     instruction): mixed path (no activation scale, M <= 4): masked nibble
-//     pairs OR-ed into fp16 exponent patterns are 1024 + q or 64 + q exactly
-//     (4 LOP3 + 1 shift per 8 codes); the producer gives each 64-input chunk
-//     of x an exact power-of-two scale into fp16; sm_100's mixed-precision FMA
-//     (fp16 x fp16 + fp32, exact product) accumulates, and each (row, chunk)
-//     sum loses the bias terms and z * sum(x) and is scaled by s16 * 2^-e in
-//     fp32.  Packed path (AWQ fold, M = 8): bf16 pairs 128 + q (mask into
-//     0x43004300) are widened to the fp32 code q - z by a mixed-precision add
-//     and packed fp32x2 FMAs multiply them with the fp32 activations;
+//   * dequantization in registers without conversion instructions.  Integer
+//     path (no activation scale, M <= 4): the producer rounds each 64-input
+//     chunk of x to integers x_i = rn(x * 2^e), e putting the chunk's largest
+//     |x| in [2^14, 2^15); two masks per code word leave the 8 codes in place
+//     as bytes (q or 16 q), and four dp4a per word and row of x (unsigned code
+//     bytes times signed high / unsigned low activation bytes, int32
+//     accumulators) give sum q x_i exactly; each (row, chunk) sum then loses
+//     z * sum x_i and is scaled by s16 * 2^-e in fp32.  Packed path (AWQ
+//     fold, M = 8): bf16 pairs 128 + q (mask into 0x43004300) are widened to
+//     the fp32 code q - z by a mixed-precision add and packed fp32x2 FMAs
+//     multiply them with the fp32 activations;
 //   * 8 lanes share a row of a tile, lane p covering inputs 64p..64p+63 of
 //     the slab; their partial sums of several rows are combined with a
 //     transposing shuffle reduction;
@@ -64,7 +66,7 @@ struct GemvParams {
   unsigned long long drain_ns;
   // Masks and exponent patterns of the code extraction, passed at run time so
   // that each extraction is one 3-register LOP3 instead of two immediate ops.
-  uint32_t lop_mask_lo, lop_mask_hi, lop_f16_1024, lop_f16_64, lop_bf16_128;
+  uint32_t lop_mask_lo, lop_bf16_128;
 };
 
 constexpr int kConsumerWarps = 8;
@@ -72,18 +74,18 @@ constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxFullTile = kTileRows * kSlabGroups * (kCodeBytesPerGroupRow + 4);
 constexpr int kLaneK = 64;                          // inputs of one row per lane
 constexpr int kChunks = kSlabK / kLaneK;            // 8 lanes per row
-constexpr int kXbChunk = kLaneK * 2 + 16;           // bf16 chunk + pad (conflict-free)
+constexpr int kXbChunk = kLaneK * 2 + 16;           // 2 activation bytes per input + pad (conflict-free)
 constexpr int kXfChunk = kLaneK * 4 + 16;           // fp32 chunk + pad
 
-template <int MP, bool MIXED>
+template <int MP, bool IDOT>
 struct StageLayout {
   static constexpr int kX = kMaxFullTile;
-  static constexpr int kXRow = kChunks * (MIXED ? kXbChunk : kXfChunk);
-  static constexpr int kXsum = kX + MP * kXRow;     // mixed: float4 [MP][8] chunk info
-  static constexpr int kBytes = kXsum + (MIXED ? MP * kChunks * 16 : 0);
+  static constexpr int kXRow = kChunks * (IDOT ? kXbChunk : kXfChunk);
+  static constexpr int kXsum = kX + MP * kXRow;     // integer path: float4 [MP][8] chunk info
+  static constexpr int kBytes = kXsum + (IDOT ? MP * kChunks * 16 : 0);
   // raw activation slot: bf16 [MP][512], then fp32 [512] of the AWQ factor
   static constexpr int kRawInv = MP * kSlabK * 2;
-  static constexpr int kRawBytes = kRawInv + (MIXED ? 0 : kSlabK * 4);
+  static constexpr int kRawBytes = kRawInv + (IDOT ? 0 : kSlabK * 4);
 };
 
 // Sum v[] over the L lanes (L = 8 or 16, lane index p) of a lane group.
@@ -129,7 +131,7 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
 }
 
 struct LopConsts {
-  uint32_t mlo, mhi, f1024, f64, b128;   // 0x000F000F 0x00F000F0 0x64006400 0x54005400 0x43004300
+  uint32_t mlo, b128;   // 0x000F000F 0x43004300
 };
 
 // Two bf16 values 128 + q of the nibble slots at bits [4i, 4i+4) and
@@ -139,33 +141,24 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i, const LopConsts&
   return and_or(w >> (4 * i), k.mlo, k.b128);
 }
 
-// acc += x_k * c_k for the 8 inputs of one (interleaved) word, with sm_100's
-// mixed-precision FMA (fp16 * fp16 + fp32, one rounding, exact product).  The
-// codes come out of 4 LOP3s as fp16 pairs of adjacent inputs: OR-ing the
-// nibble slots at bits [0,4) / [16,20) into 0x6400 (1024, unit step) gives
-// 1024 + q for inputs 0, 1; OR-ing the slots at bits [4,8) / [20,24) into
-// 0x5400 (64, step 1/16 per mantissa bit, so 1 per nibble unit) gives 64 + q
-// for inputs 2, 3; the same on w >> 8 for inputs 4, 5 and 6, 7.  xw holds the
-// activations as fp16 pairs (x0,x1) (x2,x3) (x4,x5) (x6,x7), so
-//   a0 + a1 = sum_k x_k q_k + 1024 (x0+x1+x4+x5) + 64 (x2+x3+x6+x7).
-__device__ __forceinline__ void mixed_word(uint32_t w, const uint4& xw, float& a0, float& a1,
-                                           const LopConsts& k) {
-  const uint32_t w8 = w >> 8;
-  const uint32_t ca = and_or(w, k.mlo, k.f1024);     // (1024 + q0, 1024 + q1)
-  const uint32_t cb = and_or(w, k.mhi, k.f64);       // (64 + q2, 64 + q3)
-  const uint32_t cc = and_or(w8, k.mlo, k.f1024);    // (1024 + q4, 1024 + q5)
-  const uint32_t cd = and_or(w8, k.mhi, k.f64);      // (64 + q6, 64 + q7)
-  asm("{\n\t.reg .b16 c0, c1, c2, c3, c4, c5, c6, c7, x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
-      "mov.b32 {c0, c1}, %2;\n\tmov.b32 {c2, c3}, %3;\n\t"
-      "mov.b32 {c4, c5}, %4;\n\tmov.b32 {c6, c7}, %5;\n\t"
-      "mov.b32 {x0, x1}, %6;\n\tmov.b32 {x2, x3}, %7;\n\t"
-      "mov.b32 {x4, x5}, %8;\n\tmov.b32 {x6, x7}, %9;\n\t"
-      "fma.rn.f32.f16 %0, c0, x0, %0;\n\tfma.rn.f32.f16 %1, c1, x1, %1;\n\t"
-      "fma.rn.f32.f16 %0, c2, x2, %0;\n\tfma.rn.f32.f16 %1, c3, x3, %1;\n\t"
-      "fma.rn.f32.f16 %0, c4, x4, %0;\n\tfma.rn.f32.f16 %1, c5, x5, %1;\n\t"
-      "fma.rn.f32.f16 %0, c6, x6, %0;\n\tfma.rn.f32.f16 %1, c7, x7, %1;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "r"(ca), "r"(cb), "r"(cc), "r"(cd), "r"(xw.x), "r"(xw.y), "r"(xw.z), "r"(xw.w));
+// Integer dot products of the 8 codes of one (interleaved) word with the
+// 16-bit fixed-point activations of its inputs, four bytes at a time: the
+// low nibbles masked in place are the codes of inputs 0, 4, 1, 5 as bytes,
+// the high nibbles masked in place are 16 x the codes of inputs 2, 6, 3, 7.
+// xw holds the matching activation bytes: (high bytes of inputs 0, 4, 1, 5),
+// (high bytes of 2, 6, 3, 7), then the low bytes in the same two orders.
+//   a[0] += sum q h (low nibbles), a[1] += 16 sum q h (high nibbles),
+//   a[2] += sum q l, a[3] += 16 sum q l,
+// so sum_k q_k x_k = 256 (a[0] + a[1] / 16) + a[2] + a[3] / 16, exactly.
+__device__ __forceinline__ void dp4a_word(uint32_t w, const uint4& xw, int (&a)[4]) {
+  const uint32_t lo = w & 0x0F0F0F0Fu;
+  const uint32_t hi = w & 0xF0F0F0F0u;
+  asm("dp4a.u32.s32 %0, %4, %6, %0;\n\t"
+      "dp4a.u32.s32 %1, %5, %7, %1;\n\t"
+      "dp4a.u32.u32 %2, %4, %8, %2;\n\t"
+      "dp4a.u32.u32 %3, %5, %9, %3;"
+      : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3])
+      : "r"(lo), "r"(hi), "r"(xw.x), "r"(xw.y), "r"(xw.z), "r"(xw.w));
 }
 
 // The 8 codes of one (interleaved) word as exact fp32 (q - z) pairs, in input
@@ -198,17 +191,17 @@ __device__ __forceinline__ int owner_cta(long long u, long long T, int G) {
 
 // The producer lanes' share of one activation slab: lane l holds inputs
 // 16l .. 16l+15 of the slab for every row of x (and of the AWQ factor).
-template <int MP, bool MIXED>
+template <int MP, bool IDOT>
 struct XSlice {
   uint4 xb[MP][2];
-  float4 inv[MIXED ? 1 : 4];
+  float4 inv[IDOT ? 1 : 4];
 };
 
 // Read lane l's share (inputs 16l .. 16l+15 of the slab) from a raw slot.
-template <int MP, bool MIXED>
-__device__ __forceinline__ void read_x_slice(XSlice<MP, MIXED>& xs, const uint8_t* raw,
+template <int MP, bool IDOT>
+__device__ __forceinline__ void read_x_slice(XSlice<MP, IDOT>& xs, const uint8_t* raw,
                                              const GemvParams& prm, int s, int lane) {
-  using SL = StageLayout<MP, MIXED>;
+  using SL = StageLayout<MP, IDOT>;
   const bool ok = s * kSlabK + 16 * lane < prm.g.K;   // inside the slab's groups
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
@@ -220,7 +213,7 @@ __device__ __forceinline__ void read_x_slice(XSlice<MP, MIXED>& xs, const uint8_
       xs.xb[m][1] = src[1];
     }
   }
-  if constexpr (!MIXED) {
+  if constexpr (!IDOT) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       xs.inv[q] = make_float4(1.f, 1.f, 1.f, 1.f);
@@ -230,59 +223,83 @@ __device__ __forceinline__ void read_x_slice(XSlice<MP, MIXED>& xs, const uint8_
   }
 }
 
-template <int MP, bool MIXED>
-__device__ __forceinline__ void store_x_slice(const XSlice<MP, MIXED>& xs, uint8_t* stage,
+template <int MP, bool IDOT>
+__device__ __forceinline__ void store_x_slice(const XSlice<MP, IDOT>& xs, uint8_t* stage,
                                               const GemvParams& prm, int lane) {
-  using SL = StageLayout<MP, MIXED>;
+  using SL = StageLayout<MP, IDOT>;
   const int c = lane >> 2, sub = lane & 3;      // 64-input chunk and quarter of it
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
     if (m >= prm.M) break;
     const uint32_t r[8] = {xs.xb[m][0].x, xs.xb[m][0].y, xs.xb[m][0].z, xs.xb[m][0].w,
                            xs.xb[m][1].x, xs.xb[m][1].y, xs.xb[m][1].z, xs.xb[m][1].w};
-    if constexpr (MIXED) {
-      // fp16 copy of the chunk scaled by 2^e, e chosen from the chunk's largest
-      // |x| so that it lands in [2^14, 2^15): bf16's 8-bit significands fit
-      // fp16's 11 bits, so every value within 2^-28 of the largest is exact.
+    if constexpr (IDOT) {
+      // 16-bit fixed point per 64-input chunk: x_i = rn(x * 2^e) with e chosen
+      // from the chunk's largest |x| so that it lands in [2^14, 2^15) (exact
+      // there: bf16 has 8 significant bits), every other value within half a
+      // step 2^-e.  x_i = 256 h + l is stored as signed high bytes h and
+      // unsigned low bytes l, ordered like the code bytes of an interleaved
+      // word (see dp4a_word).  A chunk holding a NaN or an infinity stores
+      // zeros and a NaN factor, so the rows it meets come out NaN.
       float xf[16];
+      bool bad = false;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         xf[2 * q] = bf16_lo(r[q]);
         xf[2 * q + 1] = bf16_hi(r[q]);
+        bad |= (r[q] & 0x7F80u) == 0x7F80u || (r[q] & 0x7F800000u) == 0x7F800000u;
       }
       float amax = 0.0f;
 #pragma unroll
       for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(xf[q]));
       amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-      const int eb = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
-      int e = (eb == 0) ? 0 : 141 - eb;            // amax * 2^e in [2^14, 2^15)
-      e = e < -126 ? -126 : (e > 126 ? 126 : e);
-      const float scale = __uint_as_float((uint32_t)(e + 127) << 23);
-      const float unscale = __uint_as_float((uint32_t)(127 - e) << 23);
-      uint32_t hw[8];
-      float sa = 0.0f, sb = 0.0f;                 // sums at the 1024- and 64-biased slots
-#pragma unroll
-      for (int wd = 0; wd < 2; ++wd) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __half lo = __float2half_rn(__fmul_rn(xf[8 * wd + 2 * i], scale));
-          const __half hi = __float2half_rn(__fmul_rn(xf[8 * wd + 2 * i + 1], scale));
-          hw[4 * wd + i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-          const float f = __half2float(lo) + __half2float(hi);
-          if (i & 1) sb += f; else sa += f;
+      bad = __shfl_xor_sync(0xFFFFFFFFu, (int)bad, 1) | bad;
+      bad = __shfl_xor_sync(0xFFFFFFFFu, (int)bad, 2) | bad;
+      int e = 0;
+      if (!bad && amax > 0.0f) {
+        int eb = (int)(__float_as_uint(amax) >> 23), pre = 0;
+        if (eb == 0) {                               // subnormal: exponent of amax * 2^64
+          eb = (int)(__float_as_uint(amax * 0x1p64f) >> 23);
+          pre = 64;
         }
+        e = 141 - eb + pre;                          // in [-113, 147]
+      }
+      // 2^-e as fp32 (subnormal above 126), and 2^e as two normal factors
+      const float unscale = bad ? __uint_as_float(0x7FC00000u)
+                            : (e <= 126 ? __uint_as_float((uint32_t)(127 - e) << 23)
+                                        : __uint_as_float(1u << (149 - e)));
+      const int e1 = e > 127 ? 64 : e;
+      const float f1 = __uint_as_float((uint32_t)(e1 + 127) << 23);
+      const float f2 = __uint_as_float((uint32_t)(e - e1 + 127) << 23);
+      int xi[16];
+      int sx = 0;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        xi[q] = bad ? 0 : __float2int_rn(__fmul_rn(__fmul_rn(xf[q], f1), f2));
+        sx += xi[q];
+      }
+      uint32_t wv[8];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int* v = xi + 8 * t;
+        // code byte order of an interleaved word: low nibbles hold inputs
+        // 0, 4, 1, 5 and high nibbles inputs 2, 6, 3, 7
+        auto hb = [](int a) { return (uint32_t)(a >> 8) & 0xFFu; };
+        auto lb = [](int a) { return (uint32_t)a & 0xFFu; };
+        wv[4 * t + 0] = hb(v[0]) | hb(v[4]) << 8 | hb(v[1]) << 16 | hb(v[5]) << 24;
+        wv[4 * t + 1] = hb(v[2]) | hb(v[6]) << 8 | hb(v[3]) << 16 | hb(v[7]) << 24;
+        wv[4 * t + 2] = lb(v[0]) | lb(v[4]) << 8 | lb(v[1]) << 16 | lb(v[5]) << 24;
+        wv[4 * t + 3] = lb(v[2]) | lb(v[6]) << 8 | lb(v[3]) << 16 | lb(v[7]) << 24;
       }
       uint4* dst = reinterpret_cast<uint4*>(stage + SL::kX + m * SL::kXRow + c * kXbChunk + sub * 32);
-      dst[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      dst[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-      sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
-      sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 2);
-      sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
-      sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 2);
+      dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+      sx += __shfl_xor_sync(0xFFFFFFFFu, sx, 1);
+      sx += __shfl_xor_sync(0xFFFFFFFFu, sx, 2);
       if (sub == 0)
         reinterpret_cast<float4*>(stage + SL::kXsum)[m * kChunks + c] =
-            make_float4(1024.0f * sa + 64.0f * sb, sa + sb, unscale, 0.0f);
+            make_float4((float)sx, unscale, 0.0f, 0.0f);
     } else {
       float4* dst = reinterpret_cast<float4*>(stage + SL::kX + m * SL::kXRow + c * kXfChunk + sub * 64);
 #pragma unroll
@@ -297,10 +314,10 @@ __device__ __forceinline__ void store_x_slice(const XSlice<MP, MIXED>& xs, uint8
 }
 
 // Bytes of shared memory one (virtual) CTA of the GEMV uses, rounded to 128.
-template <int MP, int STAGES, int RAWS, bool MIXED>
+template <int MP, int STAGES, int RAWS, bool IDOT>
 __host__ __device__ constexpr size_t gemv_team_smem() {
-  return ((size_t)STAGES * StageLayout<MP, MIXED>::kBytes +
-          (size_t)RAWS * StageLayout<MP, MIXED>::kRawBytes + (2 * STAGES + RAWS) * 8 + 16 + 127) /
+  return ((size_t)STAGES * StageLayout<MP, IDOT>::kBytes +
+          (size_t)RAWS * StageLayout<MP, IDOT>::kRawBytes + (2 * STAGES + RAWS) * 8 + 16 + 127) /
          128 * 128;
 }
 
@@ -310,12 +327,12 @@ __host__ __device__ constexpr size_t gemv_team_smem() {
 // so every team gets warps of every age: CTAs sharing an SM are not scheduled
 // evenly (the older CTA's warps win the issue slots), teams inside one CTA
 // are, and the SM's work then finishes at the same time.
-template <int MP, int JQ, int STAGES, int RAWS, int VC, bool MIXED>
+template <int MP, int JQ, int STAGES, int RAWS, int VC, bool IDOT>
 __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvParams prm) {
-  using SL = StageLayout<MP, MIXED>;
+  using SL = StageLayout<MP, IDOT>;
   extern __shared__ __align__(128) uint8_t smem_all[];
   const int team = (threadIdx.x >> 5) % VC;
-  uint8_t* smem = smem_all + team * gemv_team_smem<MP, STAGES, RAWS, MIXED>();
+  uint8_t* smem = smem_all + team * gemv_team_smem<MP, STAGES, RAWS, IDOT>();
   const Geom g = prm.g;
   uint8_t* raw_ring = smem + STAGES * SL::kBytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(raw_ring + RAWS * SL::kRawBytes);
@@ -424,9 +441,9 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
         mbar_arrive(&full_bar[st]);      // let the stage's phase complete once the copy lands
         break;
       }
-      XSlice<MP, MIXED> xs;
-      read_x_slice<MP, MIXED>(xs, raw_ring + rs * SL::kRawBytes, prm, ps, lane);
-      store_x_slice<MP, MIXED>(xs, stage, prm, lane);
+      XSlice<MP, IDOT> xs;
+      read_x_slice<MP, IDOT>(xs, raw_ring + rs * SL::kRawBytes, prm, ps, lane);
+      store_x_slice<MP, IDOT>(xs, stage, prm, lane);
       mbar_arrive(&full_bar[st]);
       ps = next_slab(ps);
       if (ps == 0) ++pb;
@@ -461,8 +478,7 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
   constexpr int V = JQ * MP;
   constexpr int kPasses = 4 / JQ;
   using GM = GroupMap<V, 8>;
-  const LopConsts lk{prm.lop_mask_lo, prm.lop_mask_hi, prm.lop_f16_1024, prm.lop_f16_64,
-                     prm.lop_bf16_128};
+  const LopConsts lk{prm.lop_mask_lo, prm.lop_bf16_128};
 
   float run[kPasses][GM::kPerLane];
 #pragma unroll
@@ -499,8 +515,8 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
       auto tile_compute = [&](auto ragged_tag) {
       constexpr bool kRagged = decltype(ragged_tag)::value;
       const bool active = !kRagged || p < 2 * gs;
-      [[maybe_unused]] float4 xinfo[MIXED ? MP : 1];   // mixed: (bias, sum x, 2^-e, -) of this lane's chunk
-      if constexpr (MIXED) {
+      [[maybe_unused]] float4 xinfo[IDOT ? MP : 1];   // integer path: (sum x_i, 2^-e, -, -) of this lane's chunk
+      if constexpr (IDOT) {
 #pragma unroll
         for (int m = 0; m < MP; ++m)
           xinfo[m] = reinterpret_cast<const float4*>(stage + SL::kXsum)[m * kChunks + p];
@@ -530,12 +546,14 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
         // for several rows of x the halves run one after the other, which
         // bounds how many activation words the compiler keeps in flight.
         constexpr int kHalfUnroll = (MP == 1) ? 2 : 1;
-        if constexpr (MIXED) {
-          float a0[JQ][MP], a1[JQ][MP];
+        if constexpr (IDOT) {
+          int acc[JQ][MP][4];
 #pragma unroll
           for (int j = 0; j < JQ; ++j)
 #pragma unroll
-            for (int m = 0; m < MP; ++m) a0[j][m] = a1[j][m] = 0.0f;
+            for (int m = 0; m < MP; ++m)
+#pragma unroll
+              for (int t = 0; t < 4; ++t) acc[j][m][t] = 0;
 #pragma unroll kHalfUnroll
           for (int hf = 0; hf < 2; ++hf) {
             uint4 c[JQ];
@@ -556,19 +574,21 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
               for (int j = 0; j < JQ; ++j) {
                 const uint32_t w = wd == 0 ? c[j].x : wd == 1 ? c[j].y : wd == 2 ? c[j].z : c[j].w;
 #pragma unroll
-                for (int m = 0; m < MP; ++m) mixed_word(w, xw[m], a0[j][m], a1[j][m], lk);
+                for (int m = 0; m < MP; ++m) dp4a_word(w, xw[m], acc[j][m]);
               }
             }
           }
           // partial of (row, m) over this lane's 64 inputs:
-          //   s16 * 2^-e * ((acc - bias) - z * sum x)
+          //   s16 * 2^-e * (sum x_i q - z * sum x_i)
 #pragma unroll
           for (int j = 0; j < JQ; ++j)
 #pragma unroll
-            for (int m = 0; m < MP; ++m)
-              v[j * MP + m] = active ? (sc[j] * xinfo[m].z) *
-                                           (((a0[j][m] + a1[j][m]) - xinfo[m].x) - zc[j] * xinfo[m].y)
+            for (int m = 0; m < MP; ++m) {
+              const int* a = acc[j][m];
+              const int t = 256 * (a[0] + (a[1] >> 4)) + a[2] + (int)((uint32_t)a[3] >> 4);
+              v[j * MP + m] = active ? (sc[j] * ((float)t - zc[j] * xinfo[m].x)) * xinfo[m].y
                                      : 0.0f;
+            }
         } else {
           float2 acc[JQ][MP];
           float cz[JQ];
@@ -717,19 +737,20 @@ struct GemvConfig {
   int teams;               // virtual CTAs per CTA
 };
 
-template <int MP, int JQ, int STAGES, int RAWS, int VC, bool MIXED>
+template <int MP, int JQ, int STAGES, int RAWS, int VC, bool IDOT>
 static GemvConfig gemv_config() {
   GemvConfig c;
-  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, RAWS, VC, MIXED>);
-  c.smem = VC * gemv_team_smem<MP, STAGES, RAWS, MIXED>();
+  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, RAWS, VC, IDOT>);
+  c.smem = VC * gemv_team_smem<MP, STAGES, RAWS, IDOT>();
   c.teams = VC;
   return c;
 }
 
 static int padded_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
-// Mixed path for M <= 4 without an activation scale; packed fp32 path for the
-// AWQ fold and for M > 4 (where one widening per code is shared by 8 rows).
+// Integer (dp4a) path for M <= 4 without an activation scale; packed fp32
+// path for the AWQ fold and for M > 4 (where one widening per code is shared
+// by 8 rows).
 // Stage counts keep two CTAs per SM where M <= 2.
 static GemvConfig pick_gemv(int M, bool awq) {
   switch (padded_m(M)) {
@@ -764,9 +785,6 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   prm.wait_ns = wait_ns;
   prm.drain_ns = 1000000000ull;
   prm.lop_mask_lo = 0x000F000Fu;
-  prm.lop_mask_hi = 0x00F000F0u;
-  prm.lop_f16_1024 = 0x64006400u;
-  prm.lop_f16_64 = 0x54005400u;
   prm.lop_bf16_128 = 0x43004300u;
 
   const GemvConfig c = pick_gemv(M, inv_s != nullptr);
