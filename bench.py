@@ -254,7 +254,7 @@ def run_ours(a, rank: int, world: int, local_rank: int):
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": elapsed_ms / a.steps,
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "int32+f32",
         "data": "synthetic",
         "config": {"workload": "llama70b_down_8192x28672_asym_g128_m1", "N": N, "K": K, "M": M,
                    "group_size": 128, "symmetric": sym, "weights": "N(0,0.015) bf16, seeded PCG64",
