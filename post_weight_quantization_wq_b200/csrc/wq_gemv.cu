@@ -795,6 +795,11 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   long long grid = (long long)num_sms * per_sm;
   const long long need = (prm.tiles + c.teams - 1) / c.teams;
   if (grid > need) grid = need;
+  // At most one team may be left without tiles; it is then team 0, ahead of
+  // every row tile.  A team without tiles among a row tile's owners would
+  // never deliver its piece of the split-K sum, so the last piece would
+  // never see the count it waits for.
+  while (grid > 1 && grid * c.teams > prm.tiles + 1) --grid;
   void* args[] = {&prm};
   return launch_pdl(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem,
                     stream);

@@ -85,6 +85,25 @@ def test_gemv_deterministic_and_workspace_reuse():
     assert int(ws[:wq._binding.WQ_WORKSPACE_COUNTER_BYTES].count_nonzero()) == 0
 
 
+@pytest.mark.parametrize("N,K", [(1, 2048), (64, 1664), (100, 3200), (128, 3584), (600, 1024)])
+def test_gemv_small_grid_finishes_every_row_tile(N, K):
+    """Tile counts one more than a multiple of three at M = 1 (three teams per
+    CTA): a grid with two teams more than tiles would leave a team without
+    tiles among a row tile's owners, and that row tile's split-K sum would
+    never be finished.  Every row must come out right and the completion
+    counters must be left at zero."""
+    import torch
+    W = inputs.weights(N, K, 0.02, seed=N + 5 * K)
+    qw, P, s, z = quantize_and_check(W, None, False)
+    ws = torch.zeros(max(wq._binding.wq_workspace_bytes(1, N, K), 16), dtype=torch.uint8,
+                     device="cuda")
+    x = inputs.activations(1, K, seed=K + 1)
+    for _ in range(2):
+        y = wq.linear(dev_bf16(x), qw, workspace=ws, path="gemv").cpu().numpy()
+        check_close(y, oracle.linear(x, P, s, z, K, sym=False), f"N={N} K={K}")
+        assert int(ws[:wq._binding.WQ_WORKSPACE_COUNTER_BYTES].count_nonzero()) == 0
+
+
 # ----------------------------------------------------------------- full sizes
 
 FULL = [(cid, li) for cid in (1, 2, 3, 5) for li in range(len(inputs.WORKLOADS[cid].linears))]
