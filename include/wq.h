@@ -235,6 +235,20 @@ wq_status wq_gemv_w4a16_static(const void* x, const float* inv_act_scale, const 
 void wq_debug_set_wait_limit_ns(unsigned long long ns);
 
 /*
+ * wq_debug_gemv_split -- test hook, not part of the stable ABI: how
+ * wq_gemv_w4a16 would split an M x N x K linear (awq != 0: with the
+ * activation factor) over a GPU with num_sms SMs holding ctas_per_sm of its
+ * CTAs each.  Writes the number of 128 x 512 tiles, the teams per CTA and the
+ * CTAs of the grid; team t of the grid's teams T owns tiles
+ * [t * tiles / T, (t + 1) * tiles / T).  Host arithmetic only (no device
+ * call, usable without a GPU).  WQ_ERR_INVALID_ARG for M outside 1..8, N < 1,
+ * K not a positive multiple of 128, num_sms or ctas_per_sm < 1, or a null
+ * output pointer.
+ */
+wq_status wq_debug_gemv_split(int M, int N, int K, int awq, int num_sms, int ctas_per_sm,
+                              long long* tiles, int* teams, long long* grid);
+
+/*
  * wq_stream_read_probe -- measurement helper with no counterpart on the
  * quantization pages: read `bytes` bytes of device memory at `buf` once, with
  * 16-byte streaming loads from every SM, and write their 32-bit XOR checksum

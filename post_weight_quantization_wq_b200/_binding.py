@@ -46,6 +46,7 @@ SIGNATURES = {
     "wq_last_device_status": (_I, [_P]),
     "wq_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "wq_stream_read_probe": (_I, [_P, _S, _P, _P]),
+    "wq_debug_gemv_split": (_I, [_I, _I, _I, _I, _I, _I, _P, _P, _P]),
 }
 
 _lock = threading.Lock()
@@ -155,6 +156,14 @@ def wq_last_device_status(stream=None) -> int:
 
 def wq_debug_set_wait_limit_ns(ns: int) -> None:
     load().wq_debug_set_wait_limit_ns(int(ns))
+
+
+def wq_debug_gemv_split(M, N, K, awq, num_sms, ctas_per_sm):
+    """(status, tiles, teams per CTA, grid CTAs) of wq_gemv_w4a16's split."""
+    tiles, teams, grid = ctypes.c_longlong(), ctypes.c_int(), ctypes.c_longlong()
+    st = load().wq_debug_gemv_split(M, N, K, int(awq), num_sms, ctas_per_sm, ctypes.byref(tiles),
+                                    ctypes.byref(teams), ctypes.byref(grid))
+    return st, tiles.value, teams.value, grid.value
 
 
 def wq_stream_read_probe(buf, nbytes, out, stream=None) -> int:

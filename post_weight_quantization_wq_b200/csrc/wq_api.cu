@@ -12,6 +12,9 @@ cudaError_t launch_quantize(const void* W, const float* awq, int N, int K, int s
 cudaError_t launch_relayout(const uint32_t* qweight, const void* scales, const void* zeros,
                             int N, int K, int sym, void* packed, cudaStream_t stream);
 size_t gemv_workspace_bytes(int M, int N, int K);
+long long gemv_grid(long long tiles, int teams, int num_sms, int ctas_per_sm);
+int gemv_teams(int M, bool awq);
+long long gemv_tiles(int N, int K);
 cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, int M, int N,
                         int K, int sym, float* y, void* workspace, int* err, int num_sms,
                         unsigned long long wait_ns, cudaStream_t stream);
@@ -300,5 +303,18 @@ wq_status wq_last_device_status(wq_stream_t stream) {
 // satisfied give up at once, which exercises the timeout path without
 // stalling the GPU.  Not part of the stable ABI.
 void wq_debug_set_wait_limit_ns(unsigned long long ns) { g_wait_ns.store(ns ? ns : 1ull); }
+
+// Test hook: how wq_gemv_w4a16 splits its tiles for a given SM count and
+// occupancy (host arithmetic only, no device call).  Not part of the stable ABI.
+wq_status wq_debug_gemv_split(int M, int N, int K, int awq, int num_sms, int ctas_per_sm,
+                              long long* tiles, int* teams, long long* grid) {
+  if (M < 1 || M > 8 || N < 1 || K < wq::kGroup || K % wq::kGroup != 0 || num_sms < 1 ||
+      ctas_per_sm < 1 || !tiles || !teams || !grid)
+    return WQ_ERR_INVALID_ARG;
+  *tiles = wq::gemv_tiles(N, K);
+  *teams = wq::gemv_teams(M, awq != 0);
+  *grid = wq::gemv_grid(*tiles, *teams, num_sms, ctas_per_sm);
+  return WQ_OK;
+}
 
 }  // extern "C"

@@ -761,6 +761,27 @@ static GemvConfig pick_gemv(int M, bool awq) {
   }
 }
 
+// CTAs of the persistent grid for `tiles` tiles with `teams` teams per CTA:
+// at most `ctas_per_sm` per SM and no more than the tiles need.  At most one
+// team may be left without tiles; it is then team 0, ahead of every row
+// tile.  A team without tiles among a row tile's owners would never deliver
+// its piece of the split-K sum, so the last piece would never see the count
+// it waits for.  Pure host arithmetic.
+long long gemv_grid(long long tiles, int teams, int num_sms, int ctas_per_sm) {
+  long long grid = (long long)num_sms * ctas_per_sm;
+  const long long need = (tiles + teams - 1) / teams;
+  if (grid > need) grid = need;
+  while (grid > 1 && grid * teams > tiles + 1) --grid;
+  return grid < 1 ? 1 : grid;
+}
+
+int gemv_teams(int M, bool awq) { return pick_gemv(M, awq).teams; }
+
+long long gemv_tiles(int N, int K) {
+  const Geom g = make_geom(N, K, 1);
+  return (long long)g.NS * g.NB;
+}
+
 size_t gemv_workspace_bytes(int M, int N, int K) {
   const Geom g = make_geom(N, K, 1);
   if (g.NS <= 1) return 0;
@@ -792,14 +813,7 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   cudaError_t e = kernel_setup(c.fn, c.smem, kGemvThreads * c.teams, &per_sm);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  long long grid = (long long)num_sms * per_sm;
-  const long long need = (prm.tiles + c.teams - 1) / c.teams;
-  if (grid > need) grid = need;
-  // At most one team may be left without tiles; it is then team 0, ahead of
-  // every row tile.  A team without tiles among a row tile's owners would
-  // never deliver its piece of the split-K sum, so the last piece would
-  // never see the count it waits for.
-  while (grid > 1 && grid * c.teams > prm.tiles + 1) --grid;
+  const long long grid = gemv_grid(prm.tiles, c.teams, num_sms, per_sm);
   void* args[] = {&prm};
   return launch_pdl(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem,
                     stream);
