@@ -161,8 +161,19 @@ size_t wq_gemm_workspace_bytes(int M, int N, int K);
  *
  *   y[m][n] = sum_g s16[n][g] * sum_{k in g} x'[m][k] * (q[n][k] - z[n][g])
  *
- * with x' = x (bf16, exact) or, when inv_act_scale is given, x'[m][k] =
- * fp32(x[m][k]) * inv_act_scale[k] (the AWQ fold, inv_act_scale = 1/s).
+ * where x' is the activation as the kernel multiplies it:
+ *   - M <= 4 without inv_act_scale (the integer path): each 64-input chunk
+ *     of a row of x is rounded to 16-bit fixed point, x' = rn(x * 2^e) * 2^-e
+ *     with e chosen so that the chunk's largest |x| lies in [2^14, 2^15)
+ *     (that value, and any value with at most 15 - (its exponent gap to the
+ *     largest) significant bits, stays exact; every other is within 2^-15 of
+ *     the chunk's largest |x|).  The codes times these integers are summed
+ *     exactly in int32 (dp4a), so the error in y is at most
+ *     2^-15 * sum_k |w_hat[n][k]| * max|x| over k's chunk.  A chunk holding a
+ *     NaN or an infinity makes every output of its row NaN.
+ *   - otherwise x' = x (bf16, exact in fp32) or, when inv_act_scale is given,
+ *     x'[m][k] = fp32(x[m][k]) * inv_act_scale[k] (the AWQ fold,
+ *     inv_act_scale = 1/s, one rounded fp32 product).
  *   x        bf16 [M][K];      inv_act_scale fp32 [K] or NULL;
  *   packed   the weight in kernel layout `layout` (from wq_pack_layout);
  *   y        fp32 [M][N] out;

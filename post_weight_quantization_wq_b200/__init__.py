@@ -137,5 +137,23 @@ def linear(x, qw: QuantizedWeight, inv_act_scale=None, out=None, workspace=None,
     return y
 
 
+def reset_workspaces(device=None) -> None:
+    """Forget the cached workspaces (of one device, or all); the next call
+    allocates a fresh zero-filled one."""
+    for key in list(_workspaces):
+        if device is None or key[0] == str(device):
+            del _workspaces[key]
+
+
 def last_device_status(stream=None) -> int:
-    return abi.wq_last_device_status(stream)
+    """Synchronize the stream and return (and clear) the device error word
+    (wq_last_device_status).  A call cut short by a bounded-wait timeout may
+    leave split-K completion counters set in its workspace, so on
+    WQ_ERR_TIMEOUT the cached workspaces of the current device are dropped:
+    later linear() calls without an explicit workspace start from zeroed
+    ones.  A caller-owned workspace must be zeroed by the caller."""
+    import torch
+    st = abi.wq_last_device_status(stream)
+    if st == abi.WQ_ERR_TIMEOUT:
+        reset_workspaces(torch.device("cuda", torch.cuda.current_device()))
+    return st

@@ -41,3 +41,32 @@ def test_wait_timeout_is_reported_and_context_stays_usable(M, path):
     y = wq.linear(xt, qw, workspace=ws, path=path).cpu().numpy()
     assert abi.wq_last_device_status() == abi.WQ_OK
     check_close(y, oracle.linear(x, P, s, z, K, sym=False), f"{path} after a timeout")
+
+
+@pytest.mark.parametrize("M,path", [(1, "gemv"), (16, "gemm")])
+def test_timeout_with_the_cached_workspace(M, path):
+    """linear() without a workspace uses one cached per (device, stream).  A
+    call cut short by a timeout may leave its completion counters set;
+    wq.last_device_status() reports the timeout and drops the cached
+    workspaces, so the next default call is correct without any manual
+    zeroing."""
+    N, K = 4096, 8192
+    W = inputs.weights(N, K, 0.015, seed=43)
+    qw, P, s, z = quantize_and_check(W, None, False)
+    x = inputs.activations(M, K, seed=44)
+    xt = dev_bf16(x)
+    wq.linear(xt, qw, path=path)                     # creates the cached workspace
+    assert wq.last_device_status() == abi.WQ_OK
+    try:
+        abi.wq_debug_set_wait_limit_ns(1)
+        for _ in range(3):
+            wq.linear(xt, qw, path=path)
+        st = wq.last_device_status()
+    finally:
+        abi.wq_debug_set_wait_limit_ns(DEFAULT_WAIT_NS)
+    assert st == abi.WQ_ERR_TIMEOUT
+    yref = oracle.linear(x, P, s, z, K, sym=False)
+    for _ in range(2):
+        y = wq.linear(xt, qw, path=path).cpu().numpy()
+        assert wq.last_device_status() == abi.WQ_OK
+        check_close(y, yref, f"{path} with the cached workspace after a timeout")

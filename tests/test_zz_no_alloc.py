@@ -6,7 +6,9 @@ wq_gemv_w4a16_static exists for callers that cannot allocate device memory
 allocation, or a captured region with a fixed memory pool): it keeps its
 split-K scratch in a static array inside the library.  Two calls in a row
 must each reproduce the workspace entry point's output within the tolerance
-the parity tests use.  This file is collected last on purpose."""
+the parity tests use (and in fact bit for bit: it is the same kernel with
+the same fixed reduction order), and a repeated call must take no device
+memory.  This file is collected last on purpose."""
 import numpy as np
 import pytest
 
@@ -51,11 +53,52 @@ def test_static_scratch_gemv_matches_workspace_gemv(N, K, M, awq):
     torch.cuda.synchronize()
     y_ref = y_ref.cpu().numpy()
 
-    for _ in range(2):
-        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    ys = [torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(2)]
+    for i, y in enumerate(ys):
+        torch.cuda.synchronize()
+        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         assert abi.wq_gemv_w4a16_static(x, inv, qw.packed, M, N, K, 128, 0, 1, y) == 0
         assert abi.wq_last_device_status() == 0
-        _close(y.cpu().numpy(), y_ref)
+        if i > 0:
+            # after the first call (which may load the kernel), a call takes
+            # no device memory at all
+            assert torch.cuda.mem_get_info()[0] == free0
+            assert torch.cuda.memory_allocated() == alloc0
+        out = y.cpu().numpy()
+        _close(out, y_ref)
+        # the same kernel with the same fixed reduction order: bit-identical
+        assert np.array_equal(out, y_ref)
+
+
+def test_static_scratch_after_a_timeout():
+    """A call cut short by a bounded-wait timeout may leave completion
+    counters set in the static array; the next call clears the ones it uses
+    itself, so it needs no help from the caller."""
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    N, K, M = 4096, 8192, 1
+    W = inputs.weights(N, K, 0.015, seed=77)
+    qw = wq.quantize(torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16))
+    x = torch.from_numpy(inputs.activations(M, K, seed=78).view(np.int16)).cuda().view(
+        torch.bfloat16)
+    ws_bytes = abi.wq_workspace_bytes(M, N, K)
+    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    y_ref = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    assert abi.wq_gemv_w4a16(x, None, qw.packed, M, N, K, 128, 0, 1, y_ref, ws, ws_bytes) == 0
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    try:
+        abi.wq_debug_set_wait_limit_ns(1)
+        for _ in range(3):
+            assert abi.wq_gemv_w4a16_static(x, None, qw.packed, M, N, K, 128, 0, 1, y) == 0
+        st = abi.wq_last_device_status()
+    finally:
+        abi.wq_debug_set_wait_limit_ns(2_000_000_000)
+    assert st == abi.WQ_ERR_TIMEOUT
+    for _ in range(2):
+        y.fill_(float("nan"))
+        assert abi.wq_gemv_w4a16_static(x, None, qw.packed, M, N, K, 128, 0, 1, y) == 0
+        assert abi.wq_last_device_status() == 0
+        assert torch.equal(y, y_ref)
 
 
 def test_static_scratch_refuses_shapes_beyond_its_size():
