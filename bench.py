@@ -43,8 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": "5c63e90f112ac7f96306ba696e1f75b1110a7b4e80f8a131603ad6991b07e199",
-               "bytes_per_launch": 124908544 + 3814400}
+NCU_TRAFFIC = {"sources_sha256": "dc88ca99b2c212b1f9f775a86df303feb326e54421843fe9827b0f7b53035210",
+               "bytes_per_launch": 124916736 + 3988992}
 
 
 def _args():
