@@ -202,6 +202,50 @@ wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* p
                         void* workspace, size_t ws_bytes, wq_stream_t stream);
 
 /*
+ * wq_gptq_quantize -- GPTQ: per-group 4-bit quantization in which the input
+ * columns are quantized one at a time in natural order and each column's
+ * rounding error is fed back into the columns not yet quantized, weighted by
+ * the inverse Hessian of the layer's calibration inputs, to minimize
+ * ||X W^T - X W_hat^T||^2 ("3.6 量化(Quantization)", section GPTQ: objective,
+ * H = 2 X X^T over the calibration inputs, update
+ * W[:, F] -= e_j / [H^-1]_jj [H^-1]_{j,F}; "推理优化中“用精度换性能“的核心技术：量化",
+ * section 四.2: columns in natural order with per-column error feedback;
+ * "大模型量化全景解析", section 六.2: damping of the Hessian).
+ *
+ *   W          bf16 [N][K]: the weight, row n = output channel.
+ *   X          bf16 [T][K]: T calibration input rows of the layer.
+ *   damp       H = 2 X^T X + damp * mean(diag(2 X^T X)) * I (0.01 is the
+ *              usual choice); must be >= 0.
+ *   qweight, scales, zeros: out, exactly the format of wq_quantize_rtn
+ *              (so wq_pack_layout and both linears take it unchanged); zeros
+ *              must be NULL iff symmetric.
+ *   workspace  device scratch of wq_gptq_workspace_bytes(T, N, K) bytes,
+ *              256-byte aligned, owned by the caller (its contents on entry
+ *              do not matter): about 8 (K^2 + T K + N K) bytes.
+ *   d_status   int32 on device, or NULL: 0 when all went well; bit 0: a
+ *              group met a non-finite weight (written as nibbles 0 with
+ *              scale and zero 0x7E00, like wq_quantize_rtn); bit 1: the
+ *              damped Hessian was not positive definite (a Cholesky pivot
+ *              <= 0; the codes are then not meaningful).
+ * Arithmetic: fp64 throughout, except that a group's scale and zero come
+ * from the RTN rules (fp32 range, IEEE fp32 divisions, fp16 RNE) applied to
+ * its 128 current weights rounded to fp32 when its first column is
+ * quantized; codes q = clamp(rint(w / s16) + z16) on the fp64 current
+ * weights.  The restricted inverses are taken from one Cholesky
+ * factorization of H with its index order reversed (H = R R^T, R upper); in
+ * exact arithmetic this is the same update.
+ * Limits: K <= WQ_GPTQ_MAX_K, 1 <= T <= WQ_GPTQ_MAX_T
+ * (WQ_ERR_UNSUPPORTED_SHAPE).  Enqueues about 4 K / 64 kernels on `stream`.
+ */
+#define WQ_GPTQ_MAX_K 32768
+#define WQ_GPTQ_MAX_T 65536
+size_t wq_gptq_workspace_bytes(int T, int N, int K);
+wq_status wq_gptq_quantize(const void* W, const void* X, int T, int N, int K, int group_size,
+                           int symmetric, double damp, uint32_t* qweight, void* scales,
+                           void* zeros, void* workspace, size_t ws_bytes, int* d_status,
+                           wq_stream_t stream);
+
+/*
  * wq_last_device_status -- synchronize `stream`, then report and clear the
  * device error word of the current GPU: WQ_ERR_TIMEOUT if a kernel's bounded
  * wait gave up since the last call (its outputs are then undefined),

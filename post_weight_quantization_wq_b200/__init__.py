@@ -82,6 +82,40 @@ def quantize(W, awq_scale=None, symmetric: bool = False, stream=None,
     return QuantizedWeight(N, K, symmetric, qweight, scales, zeros, packed, bad)
 
 
+def gptq_quantize(W, X, symmetric: bool = False, damp: float = 0.01, stream=None,
+                  workspace=None) -> QuantizedWeight:
+    """GPTQ on the GPU (wq_gptq_quantize): bf16 CUDA tensors W [N][K] and
+    calibration inputs X [T][K]; returns the same QuantizedWeight as
+    quantize(), laid out for the linears.  nonfinite_groups holds the
+    device status word (0 when all went well)."""
+    import torch
+    if getattr(W, "dim", lambda: 0)() != 2 or getattr(X, "dim", lambda: 0)() != 2:
+        raise ValueError("W [N][K] and X [T][K] must be 2-D")
+    N, K = W.shape
+    T = X.shape[0]
+    _require(W, "W", torch.bfloat16)
+    _require(X, "X", torch.bfloat16, (T, K), W.device)
+    dev = W.device
+    qweight = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+    scales = torch.empty((N, K // GROUP), dtype=torch.float16, device=dev)
+    zeros = None if symmetric else torch.empty((N, K // GROUP), dtype=torch.float16, device=dev)
+    need = abi.wq_gptq_workspace_bytes(T, N, K)
+    if need == 0:
+        raise ValueError(f"gptq_quantize: unsupported sizes T={T} N={N} K={K}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    d_status = torch.zeros(4, dtype=torch.int32, device=dev)
+    _check(abi.wq_gptq_quantize(W, X, T, N, K, GROUP, symmetric, damp, qweight, scales, zeros,
+                                workspace, workspace.numel(), d_status, stream),
+           "wq_gptq_quantize")
+    nbytes = abi.wq_packed_bytes(N, K, GROUP, symmetric, LAYOUT)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(abi.wq_pack_layout(qweight, scales, zeros, N, K, GROUP, symmetric, LAYOUT, packed,
+                              nbytes, stream), "wq_pack_layout")
+    return QuantizedWeight(N, K, symmetric, qweight, scales, zeros, packed,
+                           int(d_status[0].item()))
+
+
 _workspaces = {}
 
 

@@ -27,6 +27,8 @@ WQ_GROUP_SIZE = 128
 WQ_LAYOUT_TILED = 1
 WQ_WORKSPACE_COUNTER_BYTES = 262144
 WQ_STATIC_SCRATCH_BYTES = 8 << 20
+WQ_GPTQ_MAX_K = 32768
+WQ_GPTQ_MAX_T = 65536
 
 # name -> (restype, argtypes); the exported symbols of include/wq.h
 _P = ctypes.c_void_p
@@ -47,6 +49,9 @@ SIGNATURES = {
     "wq_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "wq_stream_read_probe": (_I, [_P, _S, _P, _P]),
     "wq_debug_gemv_split": (_I, [_I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "wq_gptq_workspace_bytes": (_S, [_I, _I, _I]),
+    "wq_gptq_quantize": (_I, [_P, _P, _I, _I, _I, _I, _I, ctypes.c_double, _P, _P, _P, _P, _S,
+                              _P, _P]),
 }
 
 _lock = threading.Lock()
@@ -168,3 +173,14 @@ def wq_debug_gemv_split(M, N, K, awq, num_sms, ctas_per_sm):
 
 def wq_stream_read_probe(buf, nbytes, out, stream=None) -> int:
     return load().wq_stream_read_probe(_ptr(buf), int(nbytes), _ptr(out), _stream(stream))
+
+
+def wq_gptq_workspace_bytes(T, N, K) -> int:
+    return load().wq_gptq_workspace_bytes(T, N, K)
+
+
+def wq_gptq_quantize(W, X, T, N, K, group_size, symmetric, damp, qweight, scales, zeros,
+                     workspace, ws_bytes, d_status, stream=None) -> int:
+    return load().wq_gptq_quantize(_ptr(W), _ptr(X), T, N, K, group_size, int(symmetric),
+                                   float(damp), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                                   _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream))

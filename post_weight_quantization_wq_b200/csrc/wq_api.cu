@@ -19,6 +19,10 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
                         int K, int sym, float* y, void* workspace, int* err, int num_sms,
                         unsigned long long wait_ns, cudaStream_t stream);
 size_t gemm_workspace_bytes(int M, int N, int K);
+size_t gptq_workspace_bytes(int T, int N, int K);
+cudaError_t launch_gptq(const void* W, const void* X, int T, int N, int K, int sym, double damp,
+                        uint32_t* qweight, void* scales, void* zeros, void* workspace,
+                        int* d_status, cudaStream_t stream);
 cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, int sym,
                         float* y, void* workspace, int* err, int num_sms,
                         unsigned long long wait_ns, cudaStream_t stream);
@@ -278,6 +282,37 @@ wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* p
   return from_cuda(wq::launch_gemm(x, packed, M, N, K, symmetric, y, workspace, d->err,
                                    d->num_sms, g_wait_ns.load(),
                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t wq_gptq_workspace_bytes(int T, int N, int K) {
+  if (check_dims(N, K, WQ_GROUP_SIZE) != WQ_OK || K > WQ_GPTQ_MAX_K || T < 1 ||
+      T > WQ_GPTQ_MAX_T)
+    return 0;
+  return wq::gptq_workspace_bytes(T, N, K);
+}
+
+wq_status wq_gptq_quantize(const void* W, const void* X, int T, int N, int K, int group_size,
+                           int symmetric, double damp, uint32_t* qweight, void* scales,
+                           void* zeros, void* workspace, size_t ws_bytes, int* d_status,
+                           wq_stream_t stream) {
+  wq_status st = check_dims(N, K, group_size);
+  if (st != WQ_OK) return st;
+  if (K > WQ_GPTQ_MAX_K || T < 1 || T > WQ_GPTQ_MAX_T) return WQ_ERR_UNSUPPORTED_SHAPE;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (!(damp >= 0.0) || damp > 1e6) return WQ_ERR_INVALID_ARG;
+  if (!W || !X || !qweight || !scales) return WQ_ERR_INVALID_ARG;
+  if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(qweight) || !aligned16(scales) ||
+      (zeros && !aligned16(zeros)))
+    return WQ_ERR_MISALIGNED;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return WQ_ERR_MISALIGNED;
+  const size_t need = wq::gptq_workspace_bytes(T, N, K);
+  if (!workspace || ws_bytes < need) return WQ_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return WQ_ERR_MISALIGNED;
+  cudaError_t e;
+  if (!device_state(&e)) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_gptq(W, X, T, N, K, symmetric, damp, qweight, scales, zeros,
+                                   workspace, d_status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 wq_status wq_last_device_status(wq_stream_t stream) {

@@ -81,6 +81,20 @@ def awq_scale_from_calibration(X: np.ndarray, alpha: float = 0.5) -> np.ndarray:
     return m.astype(np.float32)
 
 
+def correlated_calibration(T: int, K: int, seed: int, mix: float = 1.0) -> np.ndarray:
+    """bf16 calibration inputs X [T][K] with correlated features:
+    X = Z (I + mix * A / sqrt(K)), Z and A standard normal (fp32), so every
+    feature mixes in about mix^2 of the others' variance whatever K is (the
+    case the GPTQ error feedback is for; independent features would make it
+    plain RTN)."""
+    g = rng(seed)
+    Z = g.standard_normal((T, K), dtype=np.float32)
+    A = g.standard_normal((K, K), dtype=np.float32)
+    A *= np.float32(mix / math.sqrt(K))
+    A[np.diag_indices(K)] += np.float32(1.0)
+    return to_bf16_bits(Z @ A)
+
+
 @dataclass
 class Linear:
     name: str
