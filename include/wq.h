@@ -246,6 +246,91 @@ wq_status wq_gptq_quantize(const void* W, const void* X, int T, int N, int K, in
                            wq_stream_t stream);
 
 /*
+ * wq_awq_search -- the AWQ scale search: for alpha = i / n_grid, i = 0..n_grid,
+ * scale the input channels by s = s_X^alpha, quantize W diag(s) with per-group
+ * RTN (exactly wq_quantize_rtn with awq_scale = s) and measure the layer's
+ * output error on the calibration inputs X with the activations divided by
+ * s; pick the alpha with the smallest error ("3.6 量化(Quantization)",
+ * section AWQ: s = s_X^alpha with s_X the mean activation magnitude per input
+ * channel, alpha searched over [0, 1] per layer on calibration data,
+ * y = sum_j quant(s_j w_j) x_j / s_j; "后训练量化（PTQ, Post-Training
+ * Quantization）", section AWQ).
+ *
+ *   W          bf16 [N][K] weight;  X  bf16 [T][K] calibration inputs.
+ *   s_X,j      max(mean_t |X[t][j]|, 1e-8) in fp64.
+ *   s          s_X^alpha divided by its geometric mean (so prod_j s_j = 1),
+ *              computed in fp64 and rounded to fp32 (the quantizer's input).
+ *   losses     fp64 [n_grid + 1] out (device, 16-byte aligned):
+ *              ||X W^T - (X diag(s)^-1) dequant(Q(W diag(s)))^T||_F^2 in fp64
+ *              for every alpha, summed in a fixed order.
+ *   best       int32 out (device): the first index of the smallest loss.
+ *   scale_out  fp32 [K] out (device): s of the chosen alpha, ready for
+ *              wq_quantize_rtn(awq_scale = scale_out) and, as 1/s, for the
+ *              linears' inv_act_scale.
+ *   workspace  device scratch of wq_awq_search_workspace_bytes(T, N, K, n_grid)
+ *              bytes, 256-byte aligned, owned by the caller: about
+ *              8 (N K + T K + T N) + N K / 2 bytes.
+ * Limits: 1 <= T <= WQ_AWQ_MAX_T (WQ_ERR_UNSUPPORTED_SHAPE),
+ * 1 <= n_grid <= WQ_AWQ_MAX_GRID (WQ_ERR_INVALID_ARG).  Non-finite weights or
+ * scales give NaN losses.  Enqueues about 6 (n_grid + 1) kernels on `stream`.
+ */
+#define WQ_AWQ_MAX_T 65536
+#define WQ_AWQ_MAX_GRID 1000
+size_t wq_awq_search_workspace_bytes(int T, int N, int K, int n_grid);
+wq_status wq_awq_search(const void* W, const void* X, int T, int N, int K, int group_size,
+                        int symmetric, int n_grid, double* losses, float* scale_out, int* best,
+                        void* workspace, size_t ws_bytes, wq_stream_t stream);
+
+/*
+ * NVFP4: block-scaled 4-bit floating point, E2M1 elements in blocks of 16
+ * consecutive inputs with one E4M3 scale per block and one fp32 scale per
+ * tensor ("3.6 量化(Quantization)", section 数值格式: E2M1 magnitudes 0, 0.5,
+ * 1, 1.5, 2, 3, 4, 6; E4M3 with largest value 448; 16 E2M1 elements share one
+ * E4M3 scale plus one fp32 scale per tensor; section 实例演算: 4.5 bits per
+ * element).
+ *
+ * wq_nvfp4_quantize -- A bf16 [R][C] (C a multiple of 128) ->
+ *   codes         uint8 [R][C/2]: two E2M1 codes per byte, element 2i in the
+ *                 low nibble (bit 3 of a code is the sign);
+ *   block_scales  uint8 [R][C/16]: E4M3 codes;
+ *   tensor_scale  fp32 [1] (device): S = max(amax(A), 1e-8) / (6 * 448).
+ * Each step is one correctly rounded fp32 operation: sb = E4M3(amax_block /
+ * fl(6 S)) (round to nearest even, saturating at 448; a scale that rounds to
+ * 0 becomes the smallest subnormal 2^-9); q = E2M1(a / fl(E4M3(sb) S))
+ * (nearest magnitude, ties to the even code, saturating at 6, sign kept);
+ * a_hat = E2M1(q) E4M3(sb) S.  d_status (int32 on device, or NULL): the number
+ * of non-finite inputs (they are left out of amax; their codes are undefined).
+ *
+ * wq_nvfp4_packed_bytes / wq_nvfp4_pack_layout -- the weight layout the
+ * linear reads: the codes unchanged (N*K/2 bytes), then the block scales in
+ * the tensor cores' scale layout: for each tile of 128 rows t and each 64
+ * inputs kb, a 512-byte block at ((t * K/64) + kb) * 512 holding the 4 scales
+ * of row 128 t + 32 m1 + m0 at bytes m0 * 16 + m1 * 4 + (0..3) (rows past N
+ * are 0).
+ *
+ * wq_nvfp4_linear -- y fp32 [M][N] = dequant(x_q) dequant(W)^T, both operands
+ * NVFP4 (the FP4 tensor-core form): x bf16 [M][K] is quantized like the
+ * weights (its own tensor scale), then the block-scaled FP4 tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, block scales in tensor memory) accumulate in
+ * fp32, and the tensor scales are applied once per output.
+ *   packed          the weight from wq_nvfp4_pack_layout;
+ *   w_tensor_scale  fp32 [1] on device: the weight's S from wq_nvfp4_quantize;
+ *   workspace       wq_nvfp4_linear_workspace_bytes(M, N, K) bytes, 256-byte
+ *                   aligned (the quantized activations and split-K partials).
+ * M = 1..WQ_NVFP4_MAX_M.
+ */
+#define WQ_NVFP4_MAX_M 128
+wq_status wq_nvfp4_quantize(const void* A, int R, int C, uint8_t* codes, uint8_t* block_scales,
+                            float* tensor_scale, int* d_status, wq_stream_t stream);
+size_t wq_nvfp4_packed_bytes(int N, int K);
+wq_status wq_nvfp4_pack_layout(const uint8_t* codes, const uint8_t* block_scales, int N, int K,
+                               void* packed, size_t packed_bytes, wq_stream_t stream);
+size_t wq_nvfp4_linear_workspace_bytes(int M, int N, int K);
+wq_status wq_nvfp4_linear(const void* x, const void* packed, const float* w_tensor_scale, int M,
+                          int N, int K, float* y, void* workspace, size_t ws_bytes,
+                          wq_stream_t stream);
+
+/*
  * wq_last_device_status -- synchronize `stream`, then report and clear the
  * device error word of the current GPU: WQ_ERR_TIMEOUT if a kernel's bounded
  * wait gave up since the last call (its outputs are then undefined),

@@ -122,19 +122,27 @@ def _f32(v) -> float:
     return float(np.float32(v))
 
 
-def nvfp4_quantize(W, block: int = BLOCK):
+def nvfp4_tensor_scale(W) -> float:
+    """Reading F3: S = max(amax(W), 1e-8) / (6 * 448), rounded to fp32."""
+    W = np.asarray(W, np.float32)
+    amax = float(np.max(np.abs(W))) if W.size else 0.0
+    return _f32(max(amax, _f32(1e-8)) / (E2M1_MAX * E4M3_MAX))
+
+
+def nvfp4_quantize(W, block: int = BLOCK, S=None):
     """NVFP4 quantization of W [rows][cols] (blocks of ``block`` consecutive
     columns).  Returns (codes uint8 [rows][cols], one E2M1 code per byte;
     block scales uint8 [rows][cols/block], E4M3 codes; tensor scale S as an
-    fp32 value)."""
+    fp32 value).  ``S``: the tensor scale to use (default: the one of W, reading
+    F3), so rows of a larger tensor can be quantized on their own."""
     W = np.asarray(W, np.float32)
     rows, cols = W.shape
     if cols % block:
         raise ValueError("nvfp4_quantize: cols must be a multiple of the block")
     if not np.all(np.isfinite(W)):
         raise ValueError("nvfp4_quantize: non-finite weights")           # F7
-    amax = float(np.max(np.abs(W))) if W.size else 0.0
-    S = _f32(max(amax, _f32(1e-8)) / (E2M1_MAX * E4M3_MAX))             # F3
+    if S is None:
+        S = nvfp4_tensor_scale(W)                                         # F3
     S6 = _f32(E2M1_MAX * S)
     codes = np.zeros((rows, cols), np.uint8)
     scales = np.zeros((rows, cols // block), np.uint8)

@@ -116,6 +116,91 @@ def gptq_quantize(W, X, symmetric: bool = False, damp: float = 0.01, stream=None
                            int(d_status[0].item()))
 
 
+def awq_search(W, X, symmetric: bool = False, n_grid: int = 20, stream=None, workspace=None):
+    """AWQ scale search on the GPU (wq_awq_search): bf16 CUDA tensors W [N][K]
+    and calibration inputs X [T][K].  Returns a dict with the fp64 losses of
+    every alpha = i / n_grid (host numpy), the chosen index ``i`` and
+    ``alpha``, and ``s`` (fp32 CUDA tensor [K]) to pass to quantize() as
+    awq_scale (and 1/s to linear() as inv_act_scale)."""
+    import torch
+    if getattr(W, "dim", lambda: 0)() != 2 or getattr(X, "dim", lambda: 0)() != 2:
+        raise ValueError("W [N][K] and X [T][K] must be 2-D")
+    N, K = W.shape
+    T = X.shape[0]
+    _require(W, "W", torch.bfloat16)
+    _require(X, "X", torch.bfloat16, (T, K), W.device)
+    dev = W.device
+    need = abi.wq_awq_search_workspace_bytes(T, N, K, n_grid)
+    if need == 0:
+        raise ValueError(f"awq_search: unsupported sizes T={T} N={N} K={K} n_grid={n_grid}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    losses = torch.empty(n_grid + 1, dtype=torch.float64, device=dev)
+    s = torch.empty(K, dtype=torch.float32, device=dev)
+    best = torch.zeros(4, dtype=torch.int32, device=dev)
+    _check(abi.wq_awq_search(W, X, T, N, K, GROUP, symmetric, n_grid, losses, s, best, workspace,
+                             workspace.numel(), stream), "wq_awq_search")
+    i = int(best[0].item())
+    return {"losses": losses.cpu().numpy(), "i": i, "alpha": i / n_grid, "s": s}
+
+
+@dataclass
+class Nvfp4Weight:
+    """An NVFP4 weight: canonical codes / block scales / tensor scale plus the
+    layout the FP4 tensor-core linear reads."""
+    N: int
+    K: int
+    codes: "object"          # torch.uint8 [N][K/2]
+    scales: "object"         # torch.uint8 [N][K/16] (E4M3)
+    tensor_scale: "object"   # torch.float32 [1]
+    packed: "object"         # torch.uint8 [wq_nvfp4_packed_bytes]
+    nonfinite: int = 0
+
+
+def nvfp4_quantize_tensor(A, stream=None):
+    """NVFP4 codes, E4M3 block scales and the fp32 tensor scale of a bf16 CUDA
+    tensor A [R][C] (wq_nvfp4_quantize)."""
+    import torch
+    R, C = A.shape
+    _require(A, "A", torch.bfloat16)
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device=A.device)
+    scales = torch.empty((R, C // 16), dtype=torch.uint8, device=A.device)
+    S = torch.empty(4, dtype=torch.float32, device=A.device)
+    d_status = torch.zeros(4, dtype=torch.int32, device=A.device)
+    _check(abi.wq_nvfp4_quantize(A, R, C, codes, scales, S, d_status, stream), "wq_nvfp4_quantize")
+    return codes, scales, S, d_status
+
+
+def nvfp4_quantize(W, stream=None) -> Nvfp4Weight:
+    """Quantize a bf16 CUDA weight W [N][K] to NVFP4 and lay it out for
+    nvfp4_linear()."""
+    import torch
+    N, K = W.shape
+    codes, scales, S, d_status = nvfp4_quantize_tensor(W, stream)
+    nbytes = abi.wq_nvfp4_packed_bytes(N, K)
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _check(abi.wq_nvfp4_pack_layout(codes, scales, N, K, packed, nbytes, stream),
+           "wq_nvfp4_pack_layout")
+    return Nvfp4Weight(N, K, codes, scales, S, packed, int(d_status[0].item()))
+
+
+def nvfp4_linear(x, qw: Nvfp4Weight, out=None, workspace=None, stream=None):
+    """y = dequant(nvfp4(x)) dequant(W)^T as fp32 [M][N] on the FP4 tensor
+    cores (wq_nvfp4_linear); x bf16 CUDA [M][K], M <= 128."""
+    import torch
+    M, K = x.shape
+    _require(x, "x", torch.bfloat16, (M, qw.K), qw.packed.device)
+    y = out if out is not None else torch.empty((M, qw.N), dtype=torch.float32, device=x.device)
+    need = abi.wq_nvfp4_linear_workspace_bytes(M, qw.N, K)
+    if need == 0:
+        raise ValueError(f"nvfp4_linear: unsupported sizes M={M} N={qw.N} K={K}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(abi.wq_nvfp4_linear(x, qw.packed, qw.tensor_scale, M, qw.N, K, y, workspace,
+                               workspace.numel(), stream), "wq_nvfp4_linear")
+    return y
+
+
 _workspaces = {}
 
 

@@ -29,6 +29,9 @@ WQ_WORKSPACE_COUNTER_BYTES = 262144
 WQ_STATIC_SCRATCH_BYTES = 8 << 20
 WQ_GPTQ_MAX_K = 32768
 WQ_GPTQ_MAX_T = 65536
+WQ_AWQ_MAX_T = 65536
+WQ_AWQ_MAX_GRID = 1000
+WQ_NVFP4_MAX_M = 128
 
 # name -> (restype, argtypes); the exported symbols of include/wq.h
 _P = ctypes.c_void_p
@@ -50,6 +53,13 @@ SIGNATURES = {
     "wq_stream_read_probe": (_I, [_P, _S, _P, _P]),
     "wq_debug_gemv_split": (_I, [_I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "wq_gptq_workspace_bytes": (_S, [_I, _I, _I]),
+    "wq_awq_search_workspace_bytes": (_S, [_I, _I, _I, _I]),
+    "wq_nvfp4_quantize": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
+    "wq_nvfp4_packed_bytes": (_S, [_I, _I]),
+    "wq_nvfp4_pack_layout": (_I, [_P, _P, _I, _I, _P, _S, _P]),
+    "wq_nvfp4_linear_workspace_bytes": (_S, [_I, _I, _I]),
+    "wq_nvfp4_linear": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _S, _P]),
+    "wq_awq_search": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _S, _P]),
     "wq_gptq_quantize": (_I, [_P, _P, _I, _I, _I, _I, _I, ctypes.c_double, _P, _P, _P, _P, _S,
                               _P, _P]),
 }
@@ -184,3 +194,38 @@ def wq_gptq_quantize(W, X, T, N, K, group_size, symmetric, damp, qweight, scales
     return load().wq_gptq_quantize(_ptr(W), _ptr(X), T, N, K, group_size, int(symmetric),
                                    float(damp), _ptr(qweight), _ptr(scales), _ptr(zeros),
                                    _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream))
+
+
+def wq_awq_search_workspace_bytes(T, N, K, n_grid) -> int:
+    return load().wq_awq_search_workspace_bytes(T, N, K, n_grid)
+
+
+def wq_awq_search(W, X, T, N, K, group_size, symmetric, n_grid, losses, scale_out, best,
+                  workspace, ws_bytes, stream=None) -> int:
+    return load().wq_awq_search(_ptr(W), _ptr(X), T, N, K, group_size, int(symmetric), n_grid,
+                                _ptr(losses), _ptr(scale_out), _ptr(best), _ptr(workspace),
+                                ws_bytes, _stream(stream))
+
+
+def wq_nvfp4_quantize(A, R, C, codes, block_scales, tensor_scale, d_status, stream=None) -> int:
+    return load().wq_nvfp4_quantize(_ptr(A), R, C, _ptr(codes), _ptr(block_scales),
+                                    _ptr(tensor_scale), _ptr(d_status), _stream(stream))
+
+
+def wq_nvfp4_packed_bytes(N, K) -> int:
+    return load().wq_nvfp4_packed_bytes(N, K)
+
+
+def wq_nvfp4_pack_layout(codes, block_scales, N, K, packed, packed_bytes, stream=None) -> int:
+    return load().wq_nvfp4_pack_layout(_ptr(codes), _ptr(block_scales), N, K, _ptr(packed),
+                                       packed_bytes, _stream(stream))
+
+
+def wq_nvfp4_linear_workspace_bytes(M, N, K) -> int:
+    return load().wq_nvfp4_linear_workspace_bytes(M, N, K)
+
+
+def wq_nvfp4_linear(x, packed, w_tensor_scale, M, N, K, y, workspace, ws_bytes,
+                    stream=None) -> int:
+    return load().wq_nvfp4_linear(_ptr(x), _ptr(packed), _ptr(w_tensor_scale), M, N, K, _ptr(y),
+                                  _ptr(workspace), ws_bytes, _stream(stream))

@@ -20,6 +20,19 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
                         unsigned long long wait_ns, cudaStream_t stream);
 size_t gemm_workspace_bytes(int M, int N, int K);
 size_t gptq_workspace_bytes(int T, int N, int K);
+size_t awq_workspace_bytes(int T, int N, int K, int n_grid);
+cudaError_t launch_nvfp4_quantize(const void* A, int R, int C, uint8_t* codes, uint8_t* scales,
+                                  float* tensor_scale, int* d_status, int sf_atom, int num_sms,
+                                  cudaStream_t stream);
+cudaError_t launch_nvfp4_sf_relayout(const uint8_t* sf, int N, int K, uint8_t* out,
+                                     cudaStream_t stream);
+size_t nvfp4_linear_workspace_bytes(int M, int N, int K);
+cudaError_t launch_nvfp4_linear(const void* x, const uint8_t* packed, const float* w_scale, int M,
+                                int N, int K, float* y, void* workspace, int* err, int num_sms,
+                                unsigned long long wait_ns, cudaStream_t stream);
+cudaError_t launch_awq_search(const void* W, const void* X, int T, int N, int K, int sym,
+                              int n_grid, double* losses, float* s_out, int* best,
+                              void* workspace, int num_sms, cudaStream_t stream);
 cudaError_t launch_gptq(const void* W, const void* X, int T, int N, int K, int sym, double damp,
                         uint32_t* qweight, void* scales, void* zeros, void* workspace,
                         int* d_status, cudaStream_t stream);
@@ -313,6 +326,102 @@ wq_status wq_gptq_quantize(const void* W, const void* X, int T, int N, int K, in
   if (!device_state(&e)) return WQ_ERR_CUDA;
   return from_cuda(wq::launch_gptq(W, X, T, N, K, symmetric, damp, qweight, scales, zeros,
                                    workspace, d_status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t wq_awq_search_workspace_bytes(int T, int N, int K, int n_grid) {
+  if (check_dims(N, K, WQ_GROUP_SIZE) != WQ_OK || T < 1 || T > WQ_AWQ_MAX_T || n_grid < 1 ||
+      n_grid > WQ_AWQ_MAX_GRID)
+    return 0;
+  return wq::awq_workspace_bytes(T, N, K, n_grid);
+}
+
+wq_status wq_awq_search(const void* W, const void* X, int T, int N, int K, int group_size,
+                        int symmetric, int n_grid, double* losses, float* scale_out, int* best,
+                        void* workspace, size_t ws_bytes, wq_stream_t stream) {
+  wq_status st = check_dims(N, K, group_size);
+  if (st != WQ_OK) return st;
+  if (T < 1 || T > WQ_AWQ_MAX_T) return WQ_ERR_UNSUPPORTED_SHAPE;
+  if (n_grid < 1 || n_grid > WQ_AWQ_MAX_GRID) return WQ_ERR_INVALID_ARG;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (!W || !X || !losses || !scale_out || !best) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(losses) || !aligned16(scale_out) ||
+      (reinterpret_cast<uintptr_t>(best) & 3u))
+    return WQ_ERR_MISALIGNED;
+  const size_t need = wq::awq_workspace_bytes(T, N, K, n_grid);
+  if (!workspace || ws_bytes < need) return WQ_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return WQ_ERR_MISALIGNED;
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_awq_search(W, X, T, N, K, symmetric, n_grid, losses, scale_out,
+                                         best, workspace, d->num_sms,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_nvfp4_quantize(const void* A, int R, int C, uint8_t* codes, uint8_t* block_scales,
+                            float* tensor_scale, int* d_status, wq_stream_t stream) {
+  wq_status st = check_dims(R, C, WQ_GROUP_SIZE);
+  if (st != WQ_OK) return st;
+  if (!A || !codes || !block_scales || !tensor_scale) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(codes) || !aligned16(block_scales) ||
+      (reinterpret_cast<uintptr_t>(tensor_scale) & 3u) ||
+      (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)))
+    return WQ_ERR_MISALIGNED;
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_nvfp4_quantize(A, R, C, codes, block_scales, tensor_scale, d_status,
+                                             0, d->num_sms,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t wq_nvfp4_packed_bytes(int N, int K) {
+  if (check_dims(N, K, WQ_GROUP_SIZE) != WQ_OK) return 0;
+  return (size_t)N * K / 2 + (size_t)((N + 127) / 128) * (K / 64) * 512;
+}
+
+wq_status wq_nvfp4_pack_layout(const uint8_t* codes, const uint8_t* block_scales, int N, int K,
+                               void* packed, size_t packed_bytes, wq_stream_t stream) {
+  wq_status st = check_dims(N, K, WQ_GROUP_SIZE);
+  if (st != WQ_OK) return st;
+  if (!codes || !block_scales || !packed) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(block_scales) || !aligned16(packed))
+    return WQ_ERR_MISALIGNED;
+  if (packed_bytes < wq_nvfp4_packed_bytes(N, K)) return WQ_ERR_INVALID_ARG;
+  cudaError_t e;
+  if (!device_state(&e)) return WQ_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  e = cudaMemcpyAsync(packed, codes, (size_t)N * K / 2, cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_nvfp4_sf_relayout(
+      block_scales, N, K, static_cast<uint8_t*>(packed) + (size_t)N * K / 2, s));
+}
+
+size_t wq_nvfp4_linear_workspace_bytes(int M, int N, int K) {
+  if (check_dims(N, K, WQ_GROUP_SIZE) != WQ_OK || M < 1 || M > WQ_NVFP4_MAX_M) return 0;
+  return wq::nvfp4_linear_workspace_bytes(M, N, K);
+}
+
+wq_status wq_nvfp4_linear(const void* x, const void* packed, const float* w_tensor_scale, int M,
+                          int N, int K, float* y, void* workspace, size_t ws_bytes,
+                          wq_stream_t stream) {
+  wq_status st = check_dims(N, K, WQ_GROUP_SIZE);
+  if (st != WQ_OK) return st;
+  if (M < 1 || M > WQ_NVFP4_MAX_M) return WQ_ERR_UNSUPPORTED_SHAPE;
+  if (!x || !packed || !w_tensor_scale || !y) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(w_tensor_scale) & 3u))
+    return WQ_ERR_MISALIGNED;
+  const size_t need = wq::nvfp4_linear_workspace_bytes(M, N, K);
+  if (!workspace || ws_bytes < need) return WQ_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return WQ_ERR_MISALIGNED;
+  cudaError_t e;
+  DeviceState* d = device_state(&e);
+  if (!d) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_nvfp4_linear(x, static_cast<const uint8_t*>(packed), w_tensor_scale,
+                                           M, N, K, y, workspace, d->err, d->num_sms,
+                                           g_wait_ns.load(),
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 wq_status wq_last_device_status(wq_stream_t stream) {

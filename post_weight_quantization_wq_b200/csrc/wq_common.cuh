@@ -194,6 +194,25 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, void** args, size_t smem,
                        cudaStream_t stream);
 
+// Host: C(i, j) = beta * C(i, j) + alpha * sum_k A(i, k) B(k, j) in fp64 on
+// `stream`, with A(i, k) = A[i * a_i + k * a_k], B(k, j) = B[k * b_k + j * b_j]
+// and C(i, j) = C[i * ldc + j]; with lower != 0 only the 64 x 64 tiles that
+// touch the lower triangle are computed; beta == 0 never reads C.  A plain
+// tiled CUDA-core kernel (fp64 has no tensor-core path on this GPU's tcgen05
+// instructions), used by the offline calibrated quantizers.
+struct GemmF64 {
+  const double* A;
+  long long a_i, a_k;
+  const double* B;
+  long long b_k, b_j;
+  double* C;
+  long long ldc;
+  int M, N, K;
+  double alpha, beta;
+  int lower;
+};
+cudaError_t gemm_f64(const GemmF64& p, cudaStream_t stream);
+
 // Host: once per (device, kernel, dynamic smem size), raise the kernel's
 // dynamic shared-memory limit and query how many CTAs fit on one SM.  Later
 // calls only read the cache, so launches issued during stream capture make no

@@ -35,13 +35,17 @@
 //     the fp32 code q - z by a mixed-precision add and packed fp32x2 FMAs
 //     multiply them with the fp32 activations;
 //   * 8 lanes share a row of a tile, lane p covering inputs 64p..64p+63 of
-//     the slab; their partial sums of several rows are combined with a
+//     the slab; each lane accumulates its own partial sums over the tiles of
+//     a piece, and the lanes of a row are combined once per piece with a
 //     transposing shuffle reduction;
 //   * a row tile whose slabs are split between teams (only at the ends of a
-//     team's run) is finished through the workspace: each piece writes its
-//     fp32 partial, and the last piece to arrive (an atomic counter per 16
-//     rows) adds the pieces in slab order and resets the counter, so y does
-//     not depend on the order the GPU runs the teams in;
+//     team's run) is finished through the workspace: each piece stores its
+//     fp32 partial sums and moves on, and a small second kernel (launched as
+//     a programmatic dependent, so it is resident before this one ends and
+//     overlaps the next linear's first weight loads) adds the pieces in slab
+//     order, so y does not depend on the order the GPU runs the teams in.
+//     The streaming kernel itself never waits on another team: no fence,
+//     counter or partial-sum load sits on its critical path;
 //   * every wait is bounded (globaltimer): on timeout the kernel records the
 //     device error word, stops issuing copies, waits (bounded) for its copies
 //     in flight and returns.
@@ -57,7 +61,6 @@ struct GemvParams {
   const float* inv_s;      // fp32 [K] or nullptr
   float* y;                // fp32 [M][N]
   float* partials;         // fp32 [NS][MP][Npad]
-  unsigned* counters;      // one per 16 rows
   int* err;                // device error word
   Geom g;
   int M;                   // rows of x / y (<= MP)
@@ -70,19 +73,24 @@ struct GemvParams {
 };
 
 constexpr int kConsumerWarps = 8;
-constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
+// per team: 8 consumer warps, the activation producer, the weight producer
+constexpr int kGemvThreads = (kConsumerWarps + 2) * 32;
 constexpr int kMaxFullTile = kTileRows * kSlabGroups * (kCodeBytesPerGroupRow + 4);
 constexpr int kLaneK = 64;                          // inputs of one row per lane
 constexpr int kChunks = kSlabK / kLaneK;            // 8 lanes per row
 constexpr int kXbChunk = kLaneK * 2 + 16;           // 2 activation bytes per input + pad (conflict-free)
 constexpr int kXfChunk = kLaneK * 4 + 16;           // fp32 chunk + pad
 
+// A weight stage holds one tile (codes + metadata, kMaxFullTile bytes); the
+// prepared activations of a tile live in a slot of a separate ring, so a
+// stage can be refilled as soon as the consumers have its codes in registers.
 template <int MP, bool IDOT>
 struct StageLayout {
-  static constexpr int kX = kMaxFullTile;
+  static constexpr int kBytes = kMaxFullTile;       // one weight stage
+  static constexpr int kX = 0;                      // activations within an x slot
   static constexpr int kXRow = kChunks * (IDOT ? kXbChunk : kXfChunk);
   static constexpr int kXsum = kX + MP * kXRow;     // integer path: float4 [MP][8] chunk info
-  static constexpr int kBytes = kXsum + (IDOT ? MP * kChunks * 16 : 0);
+  static constexpr int kXSlot = kXsum + (IDOT ? MP * kChunks * 16 : 0);
   // raw activation slot: bf16 [MP][512], then fp32 [512] of the AWQ factor
   static constexpr int kRawInv = MP * kSlabK * 2;
   static constexpr int kRawBytes = kRawInv + (IDOT ? 0 : kSlabK * 4);
@@ -313,11 +321,47 @@ __device__ __forceinline__ void store_x_slice(const XSlice<MP, IDOT>& xs, uint8_
   }
 }
 
-// Bytes of shared memory one (virtual) CTA of the GEMV uses, rounded to 128.
-template <int MP, int STAGES, int RAWS, bool IDOT>
+// The scales (and zeros) of rows r0 + 4 j (j < JQ) for this lane's group grp
+// of the stage's tile (0 for lanes past a ragged slab's groups).
+template <int JQ>
+__device__ __forceinline__ void load_group_params(float (&sc)[JQ], float (&zc)[JQ],
+                                                  const uint8_t* meta, int gs, int sym, int r0,
+                                                  int grp, bool active) {
+#pragma unroll
+  for (int j = 0; j < JQ; ++j) {
+    const int r = r0 + 4 * j;
+    sc[j] = 0.0f;
+    zc[j] = 0.0f;
+    if (active) {
+      if (sym) {
+        sc[j] = __half2float(reinterpret_cast<const __half*>(meta)[r * gs + grp]);
+        zc[j] = 8.0f;
+      } else {
+        const __half2 sz = reinterpret_cast<const __half2*>(meta)[r * gs + grp];
+        sc[j] = __low2float(sz);
+        zc[j] = __high2float(sz);
+      }
+    }
+  }
+}
+
+// Half hf (16 bytes = 4 code words) of this lane's 64 inputs of rows r0 + 4 j.
+template <int JQ>
+__device__ __forceinline__ void load_codes(uint4 (&c)[JQ], const uint8_t* stage, int pitch, int r0,
+                                           int p, int hf, bool active) {
+#pragma unroll
+  for (int j = 0; j < JQ; ++j)
+    c[j] = active ? *reinterpret_cast<const uint4*>(stage + (r0 + 4 * j) * pitch + p * 32 + hf * 16)
+                  : make_uint4(0, 0, 0, 0);
+}
+
+// Bytes of shared memory one team of the GEMV uses, rounded to 128.
+template <int MP, int STAGES, int XR, int RAWS, bool IDOT>
 __host__ __device__ constexpr size_t gemv_team_smem() {
   return ((size_t)STAGES * StageLayout<MP, IDOT>::kBytes +
-          (size_t)RAWS * StageLayout<MP, IDOT>::kRawBytes + (2 * STAGES + RAWS) * 8 + 16 + 127) /
+          (size_t)XR * StageLayout<MP, IDOT>::kXSlot +
+          (size_t)RAWS * StageLayout<MP, IDOT>::kRawBytes + (2 * STAGES + 2 * XR + RAWS) * 8 +
+          16 + 127) /
          128 * 128;
 }
 
@@ -327,17 +371,30 @@ __host__ __device__ constexpr size_t gemv_team_smem() {
 // so every team gets warps of every age: CTAs sharing an SM are not scheduled
 // evenly (the older CTA's warps win the issue slots), teams inside one CTA
 // are, and the SM's work then finishes at the same time.
-template <int MP, int JQ, int STAGES, int RAWS, int VC, bool IDOT>
+//
+// A team's rings: STAGES weight stages (full: the tile's bytes landed; empty:
+// every consumer warp has this tile's codes and metadata in registers), XR
+// activation slots (xfull: the producer prepared the tile's activations;
+// xempty: every consumer warp is done with the tile) and RAWS raw activation
+// slots (bulk copies of x and of the AWQ factor).  Releasing a weight stage
+// before the arithmetic keeps it busy only for the copy and a register load,
+// so more of the shared memory is in flight (EARLY; it needs registers for
+// all of the lane's codes, so it is used where a lane covers one pass of
+// rows; otherwise the stage is released after the arithmetic).
+template <int MP, int JQ, int STAGES, int XR, int RAWS, int VC, bool IDOT, bool EARLY>
 __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvParams prm) {
   using SL = StageLayout<MP, IDOT>;
   extern __shared__ __align__(128) uint8_t smem_all[];
   const int team = (threadIdx.x >> 5) % VC;
-  uint8_t* smem = smem_all + team * gemv_team_smem<MP, STAGES, RAWS, IDOT>();
+  uint8_t* smem = smem_all + team * gemv_team_smem<MP, STAGES, XR, RAWS, IDOT>();
   const Geom g = prm.g;
-  uint8_t* raw_ring = smem + STAGES * SL::kBytes;
+  uint8_t* x_ring = smem + STAGES * SL::kBytes;
+  uint8_t* raw_ring = x_ring + XR * SL::kXSlot;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(raw_ring + RAWS * SL::kRawBytes);
   uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* raw_bar = empty_bar + STAGES;
+  uint64_t* xfull_bar = empty_bar + STAGES;
+  uint64_t* xempty_bar = xfull_bar + XR;
+  uint64_t* raw_bar = xempty_bar + XR;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(raw_bar + RAWS);
 
   const int warp = (threadIdx.x >> 5) / VC;     // warp index within the team
@@ -351,30 +408,72 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
 
   if (ltid == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full_bar[i], 1 + 32);           // producer's expect_tx + its 32 lanes
+      mbar_init(&full_bar[i], 1);                // producer's expect_tx
       mbar_init(&empty_bar[i], kConsumerWarps);
+    }
+    for (int i = 0; i < XR; ++i) {
+      mbar_init(&xfull_bar[i], 32);              // the producer's 32 lanes
+      mbar_init(&xempty_bar[i], kConsumerWarps);
     }
     for (int i = 0; i < RAWS; ++i) mbar_init(&raw_bar[i], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  // Rows of x beyond M are never written: zero every stage's activation area once.
-  for (int st = 0; st < STAGES; ++st)
-    for (int i = ltid; i < (SL::kBytes - SL::kX) / 16; i += kGemvThreads)
-      reinterpret_cast<uint4*>(smem + st * SL::kBytes + SL::kX)[i] = make_uint4(0, 0, 0, 0);
+  // Rows of x beyond M are never written: zero every activation slot once.
+  for (int i = ltid; i < XR * SL::kXSlot / 16; i += kGemvThreads)
+    reinterpret_cast<uint4*>(x_ring)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
   // Programmatic dependent launch: the next kernel in the stream may start
   // as soon as SMs free up (it waits for this grid before it touches
   // anything this grid writes).
   griddep_launch_dependents();
 
+  if (warp == kConsumerWarps + 1) {
+    // ---------------------------------------------------------- weight producer
+    // Every weight tile goes out as soon as its stage is free.  The first
+    // STAGES tiles do not depend on the previous kernel in the stream (no
+    // kernel of this library writes weights): they go out at once, so they
+    // stream in while that kernel finishes.
+    int wb = (int)(t0 / g.NS), ws = (int)(t0 % g.NS);
+    int issued = 0;
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % STAGES;
+      if (i >= STAGES) {
+        ok = mbar_wait_bounded(&empty_bar[st], ((i / STAGES) - 1) & 1, prm.wait_ns);
+        ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
+        if (!ok) break;
+      }
+      if (lane == 0) {
+        const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, ws));
+        mbar_arrive_expect_tx(&full_bar[st], tbytes);
+        bulk_copy_g2s(smem + st * SL::kBytes, prm.packed + tile_offset(g, ws, wb), tbytes,
+                      &full_bar[st]);
+      }
+      issued = i + 1;
+      if (++ws == g.NS) { ws = 0; ++wb; }
+    }
+    if (!ok && lane == 0) {
+      atomicOr(prm.err, kDevErrTimeout);
+      *abort_flag = 1;
+    }
+    if (lane == 0 && *abort_flag) {
+      // Wait (bounded) for every copy still in flight before the CTA exits.
+      for (int st = 0; st < STAGES && st < issued; ++st) {
+        const int uses = (issued - 1 - st) / STAGES + 1;   // copies issued on stage st
+        mbar_wait_bounded(&full_bar[st], (uses - 1) & 1, prm.drain_ns);
+      }
+    }
+    return;
+  }
+
   if (warp == kConsumerWarps) {
-    // ---------------------------------------------------------------- producer
+    // ------------------------------------------------------ activation producer
     // The raw activation slab (and AWQ factor) of tile i is bulk-copied into
     // raw slot i % RAWS, RAWS tiles ahead of its use, so the slab is already
-    // in shared memory when the producer converts it into tile i's stage.
-    int issued = 0, raw_issued = 0;
-    int pb = (int)(t0 / g.NS), ps = (int)(t0 % g.NS), pf = ps;
+    // in shared memory when it is prepared in activation slot i % XR.
+    int raw_issued = 0;
+    int ps = (int)(t0 % g.NS), pf = ps;
     auto next_slab = [&](int v) { return v + 1 == g.NS ? 0 : v + 1; };
     auto issue_raw = [&](int slot, int slab) {       // lane 0 only
       uint8_t* dst = raw_ring + slot * SL::kRawBytes;
@@ -386,22 +485,7 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
                       &raw_bar[slot]);
       if (ib) bulk_copy_g2s(dst + SL::kRawInv, prm.inv_s + slab * kSlabK, ib, &raw_bar[slot]);
     };
-    // The first STAGES weight tiles do not depend on the previous kernel in
-    // the stream (no kernel of this library writes weights): they go out
-    // before the wait for it, so they stream in while that kernel finishes.
-    const int early = ntiles < STAGES ? ntiles : STAGES;
-    if (lane == 0) {
-      int eb = pb, es = ps;
-      for (int k = 0; k < early; ++k) {
-        const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, es));
-        mbar_arrive_expect_tx(&full_bar[k], tbytes);
-        bulk_copy_g2s(smem + k * SL::kBytes, prm.packed + tile_offset(g, es, eb), tbytes,
-                      &full_bar[k]);
-        es = next_slab(es);
-        if (es == 0) ++eb;
-      }
-    }
-    griddep_wait();                      // x, y and the workspace may belong to it
+    griddep_wait();                      // x may belong to the previous kernel
     if (lane == 0)
       for (int r = 0; r < RAWS && r < ntiles; ++r) {
         issue_raw(r, pf);
@@ -410,11 +494,15 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
     raw_issued = ntiles < RAWS ? ntiles : RAWS;
     pf = __shfl_sync(0xFFFFFFFFu, pf, 0);
     for (int i = 0; i < ntiles; ++i) {
-      const int st = i % STAGES;
+      const int xs = i % XR;
       const int rs = i % RAWS;
       bool ok = true;
-      if (i >= STAGES) ok = mbar_wait_bounded(&empty_bar[st], ((i / STAGES) - 1) & 1, prm.wait_ns);
+      if (i >= XR) ok = mbar_wait_bounded(&xempty_bar[xs], ((i / XR) - 1) & 1, prm.wait_ns);
       ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
+      if (ok) {
+        ok = mbar_wait_bounded(&raw_bar[rs], (i / RAWS) & 1, prm.wait_ns);
+        ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
+      }
       if (!ok) {
         if (lane == 0) {
           atomicOr(prm.err, kDevErrTimeout);
@@ -422,31 +510,11 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
         }
         break;
       }
-      // The weight tile goes out as soon as its stage is free; the
-      // activation slab it is used with is converted while it streams in.
-      uint8_t* stage = smem + st * SL::kBytes;
-      if (lane == 0 && i >= early) {
-        const uint32_t tbytes = (uint32_t)tile_bytes(g, slab_groups(g, ps));
-        mbar_arrive_expect_tx(&full_bar[st], tbytes);
-        bulk_copy_g2s(stage, prm.packed + tile_offset(g, ps, pb), tbytes, &full_bar[st]);
-      }
-      issued = i + 1;
-      ok = mbar_wait_bounded(&raw_bar[rs], (i / RAWS) & 1, prm.wait_ns);
-      ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
-      if (!ok) {
-        if (lane == 0) {
-          atomicOr(prm.err, kDevErrTimeout);
-          *abort_flag = 1;
-        }
-        mbar_arrive(&full_bar[st]);      // let the stage's phase complete once the copy lands
-        break;
-      }
-      XSlice<MP, IDOT> xs;
-      read_x_slice<MP, IDOT>(xs, raw_ring + rs * SL::kRawBytes, prm, ps, lane);
-      store_x_slice<MP, IDOT>(xs, stage, prm, lane);
-      mbar_arrive(&full_bar[st]);
+      XSlice<MP, IDOT> xsl;
+      read_x_slice<MP, IDOT>(xsl, raw_ring + rs * SL::kRawBytes, prm, ps, lane);
+      store_x_slice<MP, IDOT>(xsl, x_ring + xs * SL::kXSlot, prm, lane);
+      mbar_arrive(&xfull_bar[xs]);
       ps = next_slab(ps);
-      if (ps == 0) ++pb;
       __syncwarp();                      // every lane has read raw slot rs
       if (i + RAWS < ntiles) {
         if (lane == 0) {
@@ -458,11 +526,6 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
       }
     }
     if (lane == 0 && *abort_flag) {
-      // Wait (bounded) for every copy still in flight before the CTA exits.
-      for (int st = 0; st < STAGES && st < issued; ++st) {
-        const int uses = (issued - 1 - st) / STAGES + 1;   // copies issued on stage st
-        mbar_wait_bounded(&full_bar[st], (uses - 1) & 1, prm.drain_ns);
-      }
       for (int r = 0; r < RAWS && r < raw_issued; ++r) {
         const int uses = (raw_issued - 1 - r) / RAWS + 1;
         mbar_wait_bounded(&raw_bar[r], (uses - 1) & 1, prm.drain_ns);
@@ -480,11 +543,14 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
   using GM = GroupMap<V, 8>;
   const LopConsts lk{prm.lop_mask_lo, prm.lop_bf16_128};
 
-  float run[kPasses][GM::kPerLane];
+  // Each lane keeps its own partial sums (its 64-input chunk of every tile of
+  // the current piece) of the V (row, x row) pairs of each pass; the lanes of
+  // a row are combined once, at the end of the piece.
+  float part[kPasses][V];
 #pragma unroll
   for (int a = 0; a < kPasses; ++a)
 #pragma unroll
-    for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[a][i2] = 0.0f;
+    for (int i2 = 0; i2 < V; ++i2) part[a][i2] = 0.0f;
   int piece_s0 = -1;                // first slab of the current row tile in this CTA
   bool aborted = false;
   int b = (int)(t0 / g.NS), s = (int)(t0 % g.NS) - 1;
@@ -493,6 +559,7 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
     if (++s == g.NS) { s = 0; ++b; }
     const int gs = slab_groups(g, s);
     const int st = i % STAGES;
+    const int xs = i % XR;
     if (piece_s0 < 0) piece_s0 = s;
 
     if (!aborted) {
@@ -510,42 +577,54 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
       const uint8_t* meta = stage + kTileRows * gs * kCodeBytesPerGroupRow;
       const int pitch = gs * kCodeBytesPerGroupRow;
       const int grp = p >> 1;
-      // Full slabs (all but possibly the last) take a predicate-free copy of
-      // the compute; in a ragged last slab lanes past its groups sit out.
-      auto tile_compute = [&](auto ragged_tag) {
-      constexpr bool kRagged = decltype(ragged_tag)::value;
-      const bool active = !kRagged || p < 2 * gs;
+      const bool active = p < 2 * gs;            // full slabs: always; a ragged last slab: its groups
+      // 1. EARLY: this lane's codes and group parameters of the tile into
+      //    registers, then the weight stage goes back to the producer
+      constexpr int kPI = EARLY ? kPasses : 1;   // passes whose codes are held at once
+      uint4 cw[kPI][2][JQ];
+      float scv[kPI][JQ], zcv[kPI][JQ];
+      if constexpr (EARLY) {
+#pragma unroll
+        for (int pass = 0; pass < kPasses; ++pass) {
+          load_group_params<JQ>(scv[pass], zcv[pass], meta, gs, g.sym, warp * 16 + 4 * pass * JQ + rq,
+                                grp, active);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+            load_codes<JQ>(cw[pass][hf], stage, pitch, warp * 16 + 4 * pass * JQ + rq, p, hf,
+                           active);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[st]);
+      }
+      // 2. the tile's prepared activations
+      bool ok = mbar_wait_bounded(&xfull_bar[xs], (i / XR) & 1, prm.wait_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) {
+        if (lane == 0) atomicOr(prm.err, kDevErrTimeout);
+        *abort_flag = 1;
+        aborted = true;
+      }
+      if (!aborted) {
+      const uint8_t* xslot = x_ring + xs * SL::kXSlot;
       [[maybe_unused]] float4 xinfo[IDOT ? MP : 1];   // integer path: (sum x_i, 2^-e, -, -) of this lane's chunk
       if constexpr (IDOT) {
 #pragma unroll
         for (int m = 0; m < MP; ++m)
-          xinfo[m] = reinterpret_cast<const float4*>(stage + SL::kXsum)[m * kChunks + p];
+          xinfo[m] = reinterpret_cast<const float4*>(xslot + SL::kXsum)[m * kChunks + p];
       }
 
-#pragma unroll 1
+      constexpr int kPassUnroll = kPasses;
+      // A lane's 64 inputs of a row are two 16-byte halves of 4 words each; for
+      // several rows of x (release after the arithmetic) the passes and halves
+      // run one after the other, which bounds the registers in flight.
+      constexpr int kHalfUnroll = (MP == 1) ? 2 : 1;
+#pragma unroll kPassUnroll
       for (int pass = 0; pass < kPasses; ++pass) {
-        float sc[JQ], zc[JQ];
-#pragma unroll
-        for (int j = 0; j < JQ; ++j) {
-          const int r = warp * 16 + 4 * (pass * JQ + j) + rq;
-          sc[j] = 0.0f;
-          zc[j] = 0.0f;
-          if (active) {
-            if (g.sym) {
-              sc[j] = __half2float(reinterpret_cast<const __half*>(meta)[r * gs + grp]);
-              zc[j] = 8.0f;
-            } else {
-              const __half2 sz = reinterpret_cast<const __half2*>(meta)[r * gs + grp];
-              sc[j] = __low2float(sz);
-              zc[j] = __high2float(sz);
-            }
-          }
-        }
+        const int pi = EARLY ? pass : 0;
+        if constexpr (!EARLY)
+          load_group_params<JQ>(scv[0], zcv[0], meta, gs, g.sym, warp * 16 + 4 * pass * JQ + rq,
+                                grp, active);
         float v[V];
-        // The lane's 64 inputs of a row are two 16-byte halves of 4 words each;
-        // for several rows of x the halves run one after the other, which
-        // bounds how many activation words the compiler keeps in flight.
-        constexpr int kHalfUnroll = (MP == 1) ? 2 : 1;
         if constexpr (IDOT) {
           int acc[JQ][MP][4];
 #pragma unroll
@@ -557,18 +636,18 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
 #pragma unroll kHalfUnroll
           for (int hf = 0; hf < 2; ++hf) {
             uint4 c[JQ];
+            if constexpr (EARLY) {
 #pragma unroll
-            for (int j = 0; j < JQ; ++j) {
-              const int r = warp * 16 + 4 * (pass * JQ + j) + rq;
-              c[j] = active ? *reinterpret_cast<const uint4*>(stage + r * pitch + p * 32 + hf * 16)
-                            : make_uint4(0, 0, 0, 0);
+              for (int j = 0; j < JQ; ++j) c[j] = cw[pi][hf][j];
+            } else {
+              load_codes<JQ>(c, stage, pitch, warp * 16 + 4 * pass * JQ + rq, p, hf, active);
             }
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) {
               uint4 xw[MP];
 #pragma unroll
               for (int m = 0; m < MP; ++m)
-                xw[m] = *reinterpret_cast<const uint4*>(stage + SL::kX + m * SL::kXRow +
+                xw[m] = *reinterpret_cast<const uint4*>(xslot + SL::kX + m * SL::kXRow +
                                                         p * kXbChunk + 16 * (4 * hf + wd));
 #pragma unroll
               for (int j = 0; j < JQ; ++j) {
@@ -586,7 +665,8 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
             for (int m = 0; m < MP; ++m) {
               const int* a = acc[j][m];
               const int t = 256 * (a[0] + (a[1] >> 4)) + a[2] + (int)((uint32_t)a[3] >> 4);
-              v[j * MP + m] = active ? (sc[j] * ((float)t - zc[j] * xinfo[m].x)) * xinfo[m].y
+              v[j * MP + m] = active ? (scv[pi][j] * ((float)t - zcv[pi][j] * xinfo[m].x)) *
+                                           xinfo[m].y
                                      : 0.0f;
             }
         } else {
@@ -594,18 +674,18 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
           float cz[JQ];
 #pragma unroll
           for (int j = 0; j < JQ; ++j) {
-            cz[j] = -(128.0f + zc[j]);
+            cz[j] = -(128.0f + zcv[pi][j]);
 #pragma unroll
             for (int m = 0; m < MP; ++m) acc[j][m] = make_float2(0.0f, 0.0f);
           }
 #pragma unroll kHalfUnroll
           for (int hf = 0; hf < 2; ++hf) {
             uint4 c[JQ];
+            if constexpr (EARLY) {
 #pragma unroll
-            for (int j = 0; j < JQ; ++j) {
-              const int r = warp * 16 + 4 * (pass * JQ + j) + rq;
-              c[j] = active ? *reinterpret_cast<const uint4*>(stage + r * pitch + p * 32 + hf * 16)
-                            : make_uint4(0, 0, 0, 0);
+              for (int j = 0; j < JQ; ++j) c[j] = cw[pi][hf][j];
+            } else {
+              load_codes<JQ>(c, stage, pitch, warp * 16 + 4 * pass * JQ + rq, p, hf, active);
             }
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) {
@@ -613,7 +693,7 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
 #pragma unroll
               for (int m = 0; m < MP; ++m) {
                 const float4* xp = reinterpret_cast<const float4*>(
-                    stage + SL::kX + m * SL::kXRow + p * kXfChunk + 32 * (4 * hf + wd));
+                    xslot + SL::kX + m * SL::kXRow + p * kXfChunk + 32 * (4 * hf + wd));
                 const float4 lo = xp[0], hi = xp[1];
                 xv[m][0] = make_float2(lo.x, lo.y);
                 xv[m][1] = make_float2(lo.z, lo.w);
@@ -642,23 +722,30 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
           for (int j = 0; j < JQ; ++j)
 #pragma unroll
             for (int m = 0; m < MP; ++m)
-              v[j * MP + m] = active ? sc[j] * (acc[j][m].x + acc[j][m].y) : 0.0f;
+              v[j * MP + m] = active ? scv[pi][j] * (acc[j][m].x + acc[j][m].y) : 0.0f;
         }
-        group_transpose_reduce<V, 8>(v, p);
 #pragma unroll
-        for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[pass][i2] += v[i2];
+        for (int i2 = 0; i2 < V; ++i2) part[pass][i2] += v[i2];
       }
-      };
-      if (gs == kSlabGroups) tile_compute(std::false_type{});
-      else tile_compute(std::true_type{});
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[st]);
+      if (lane == 0) {
+        if constexpr (!EARLY) mbar_arrive(&empty_bar[st]);
+        mbar_arrive(&xempty_bar[xs]);
+      }
+      }
     }
 
     // ---- end of this CTA's piece of row tile b: write y or a partial
     const bool piece_end = (s == g.NS - 1) || (i == ntiles - 1);
     if (piece_end) {
       const bool whole = (piece_s0 == 0) && (s == g.NS - 1);
+      float run[kPasses][GM::kPerLane];
+#pragma unroll
+      for (int pass = 0; pass < kPasses; ++pass) {
+        group_transpose_reduce<V, 8>(part[pass], p);
+#pragma unroll
+        for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[pass][i2] = part[pass][i2];
+      }
       if (!aborted && GM::writer(p)) {
 #pragma unroll
         for (int pass = 0; pass < kPasses; ++pass)
@@ -677,56 +764,49 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
             }
           }
       }
-      if (!whole) {
-        __threadfence();
-        __syncwarp();
-        const long long ub = (long long)b * g.NS;
-        const int c_first = owner_cta(ub, prm.tiles, G);
-        const int c_last = owner_cta(ub + g.NS - 1, prm.tiles, G);
-        unsigned prev = 0;
-        unsigned* ctr = prm.counters + (size_t)b * (kTileRows / kRowsPerCounter) + warp;
-        if (lane == 0) prev = atomicAdd(ctr, 1u);
-        prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-        if (prev == (unsigned)(c_last - c_first)) {
-          // Last piece: add all pieces in slab order, reset the counter.
-          __threadfence();
-          if (!aborted) {
-            for (int e = lane; e < kRowsPerCounter * prm.M; e += 32) {
-              const int n = b * kTileRows + warp * kRowsPerCounter + (e % kRowsPerCounter);
-              const int m = e / kRowsPerCounter;
-              // the pieces' partials, eight loads in flight at a time, added in
-              // slab order
-              float tot = 0.0f;
-              int c2 = c_first;
-              for (; c2 + 7 <= c_last; c2 += 8) {
-                float v8[8];
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                  const long long tc = (long long)(c2 + t) * prm.tiles / G;
-                  const int sa = (int)((tc > ub ? tc : ub) - ub);
-                  v8[t] = __ldcg(prm.partials + ((size_t)sa * MP + m) * g.Npad + n);
-                }
-#pragma unroll
-                for (int t = 0; t < 8; ++t) tot += v8[t];
-              }
-              for (; c2 <= c_last; ++c2) {
-                const long long tc = (long long)c2 * prm.tiles / G;
-                const int sa = (int)((tc > ub ? tc : ub) - ub);
-                tot += __ldcg(prm.partials + ((size_t)sa * MP + m) * g.Npad + n);
-              }
-              if (n < g.N) prm.y[(size_t)m * g.N + n] = tot;
-            }
-          }
-          if (lane == 0) *ctr = 0u;
-        }
-      }
 #pragma unroll
       for (int a = 0; a < kPasses; ++a)
 #pragma unroll
-        for (int i2 = 0; i2 < GM::kPerLane; ++i2) run[a][i2] = 0.0f;
+        for (int i2 = 0; i2 < V; ++i2) part[a][i2] = 0.0f;
       piece_s0 = -1;
     }
   }
+}
+
+// ------------------------------------------------------------------ finish
+
+struct FinishParams {
+  const float* partials;   // fp32 [NS][MP][Npad]
+  float* y;
+  int N, M, MP, NS, Npad, G;
+  long long tiles;
+};
+
+// y[m][n] of every row tile whose slabs were split between teams: the sum of
+// its pieces' partials in slab order (piece c of the row tile starts at slab
+// max(t0(c), b NS) - b NS).  One thread per output.  Rows of row tiles held
+// by one team were written by the streaming kernel and are left alone.
+__global__ void __launch_bounds__(256) gemv_finish_kernel(const FinishParams f) {
+  griddep_launch_dependents();
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= (long long)f.M * f.N) {
+    griddep_wait();
+    return;
+  }
+  const int m = (int)(e / f.N), n = (int)(e % f.N);
+  const int b = n / kTileRows;
+  const long long ub = (long long)b * f.NS;
+  const int c_first = owner_cta(ub, f.tiles, f.G);
+  const int c_last = owner_cta(ub + f.NS - 1, f.tiles, f.G);
+  griddep_wait();                    // the streaming kernel's partials are complete
+  if (c_first == c_last) return;
+  float tot = 0.0f;
+  for (int c2 = c_first; c2 <= c_last; ++c2) {
+    const long long tc = (long long)c2 * f.tiles / f.G;
+    const int sa = (int)((tc > ub ? tc : ub) - ub);
+    tot += __ldcg(f.partials + ((size_t)sa * f.MP + m) * f.Npad + n);
+  }
+  f.y[(size_t)m * f.N + n] = tot;
 }
 
 // ------------------------------------------------------------------ launcher
@@ -737,11 +817,12 @@ struct GemvConfig {
   int teams;               // virtual CTAs per CTA
 };
 
-template <int MP, int JQ, int STAGES, int RAWS, int VC, bool IDOT>
+template <int MP, int JQ, int STAGES, int XR, int RAWS, int VC, bool IDOT, bool EARLY>
 static GemvConfig gemv_config() {
   GemvConfig c;
-  c.fn = reinterpret_cast<const void*>(&gemv_w4a16_kernel<MP, JQ, STAGES, RAWS, VC, IDOT>);
-  c.smem = VC * gemv_team_smem<MP, STAGES, RAWS, IDOT>();
+  c.fn = reinterpret_cast<const void*>(
+      &gemv_w4a16_kernel<MP, JQ, STAGES, XR, RAWS, VC, IDOT, EARLY>);
+  c.smem = VC * gemv_team_smem<MP, STAGES, XR, RAWS, IDOT>();
   c.teams = VC;
   return c;
 }
@@ -750,14 +831,18 @@ static int padded_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
 // Integer (dp4a) path for M <= 4 without an activation scale; packed fp32
 // path for the AWQ fold and for M > 4 (where one widening per code is shared
-// by 8 rows).
-// Stage counts keep two CTAs per SM where M <= 2.
+// by 8 rows).  Teams x (weight stages, activation slots, raw slots) fill the
+// shared memory of one CTA per SM; two teams keep the registers for a tile's
+// codes held between the stage release and the arithmetic.
 static GemvConfig pick_gemv(int M, bool awq) {
   switch (padded_m(M)) {
-    case 1: return awq ? gemv_config<1, 4, 2, 2, 2, false>() : gemv_config<1, 4, 2, 3, 3, true>();
-    case 2: return awq ? gemv_config<2, 2, 4, 2, 1, false>() : gemv_config<2, 2, 2, 4, 2, true>();
-    case 4: return awq ? gemv_config<4, 2, 4, 2, 1, false>() : gemv_config<4, 2, 4, 3, 1, true>();
-    default: return gemv_config<8, 2, 3, 2, 1, false>();
+    case 1: return awq ? gemv_config<1, 4, 3, 2, 2, 2, false, true>()
+                       : gemv_config<1, 2, 3, 3, 2, 2, true, true>();
+    case 2: return awq ? gemv_config<2, 2, 5, 2, 2, 1, false, false>()
+                       : gemv_config<2, 2, 3, 2, 3, 2, true, false>();
+    case 4: return awq ? gemv_config<4, 2, 5, 2, 2, 1, false, false>()
+                       : gemv_config<4, 2, 5, 2, 3, 1, true, false>();
+    default: return gemv_config<8, 2, 5, 2, 2, 1, false, false>();
   }
 }
 
@@ -797,7 +882,6 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   prm.x = static_cast<const uint16_t*>(x);
   prm.inv_s = inv_s;
   prm.y = y;
-  prm.counters = static_cast<unsigned*>(workspace);
   prm.partials = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes)
                            : nullptr;
   prm.err = err;
@@ -815,8 +899,22 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   const long long grid = gemv_grid(prm.tiles, c.teams, num_sms, per_sm);
   void* args[] = {&prm};
-  return launch_pdl(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem,
-                    stream);
+  e = launch_pdl(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem, stream);
+  if (e != cudaSuccess || prm.g.NS <= 1) return e;
+  FinishParams f;
+  f.partials = prm.partials;
+  f.y = y;
+  f.N = N;
+  f.M = M;
+  f.MP = padded_m(M);
+  f.NS = prm.g.NS;
+  f.Npad = prm.g.Npad;
+  f.G = (int)(grid * c.teams);
+  f.tiles = prm.tiles;
+  void* fargs[] = {&f};
+  const long long outs = (long long)M * N;
+  return launch_pdl(reinterpret_cast<const void*>(&gemv_finish_kernel),
+                    dim3((unsigned)((outs + 255) / 256)), dim3(256), fargs, 0, stream);
 }
 
 }  // namespace wq

@@ -36,21 +36,7 @@
 namespace wq {
 
 // ------------------------------------------------------------------ fp64 GEMM
-// C(i, j) = beta * C(i, j) + alpha * sum_k A(i, k) B(k, j) with
-// A(i, k) = A[i * a_i + k * a_k], B(k, j) = B[k * b_k + j * b_j],
-// C(i, j) = C[i * ldc + j].  With lower != 0 only tiles that touch the lower
-// triangle (tile column <= tile row) are computed.  beta == 0 never reads C.
-struct GemmF64 {
-  const double* A;
-  long long a_i, a_k;
-  const double* B;
-  long long b_k, b_j;
-  double* C;
-  long long ldc;
-  int M, N, K;
-  double alpha, beta;
-  int lower;
-};
+// (GemmF64 is declared in wq_common.cuh.)
 
 constexpr int kFB = 64;       // tile rows and columns
 constexpr int kFK = 16;       // k per smem stage
@@ -130,7 +116,7 @@ __global__ void __launch_bounds__(256) gemm_f64_kernel(const GemmF64 p) {
   }
 }
 
-static cudaError_t gemm_f64(const GemmF64& p, cudaStream_t stream) {
+cudaError_t gemm_f64(const GemmF64& p, cudaStream_t stream) {
   if (p.M <= 0 || p.N <= 0) return cudaSuccess;
   dim3 grid((p.N + kFB - 1) / kFB, (p.M + kFB - 1) / kFB);
   gemm_f64_kernel<<<grid, 256, 0, stream>>>(p);

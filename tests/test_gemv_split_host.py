@@ -48,10 +48,10 @@ def test_split_leaves_no_idle_team_inside_a_row_tile(M, awq):
 
 
 def test_split_of_the_headline_linear():
-    """8192 x 28672 at M = 1: 3,584 tiles over one CTA per SM of 148, three
-    teams each (444 teams, 8 or 9 tiles each)."""
+    """8192 x 28672 at M = 1: 3,584 tiles over one CTA per SM of 148, two
+    teams each (296 teams, 12 or 13 tiles each)."""
     st, tiles, teams, grid = abi.wq_debug_gemv_split(1, 8192, 28672, 0, 148, 1)
-    assert (st, tiles, teams, grid) == (abi.WQ_OK, 3584, 3, 148)
+    assert (st, tiles, teams, grid) == (abi.WQ_OK, 3584, 2, 148)
 
 
 @pytest.mark.parametrize("args", [(0, 1, 128, 0, 148, 1), (9, 1, 128, 0, 148, 1),
