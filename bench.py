@@ -39,6 +39,7 @@ METRIC = "W4A16 G128 GEMV µs/linear and achieved HBM TB/s vs B200 peak at M=1"
 UNIT = "us/linear"
 WORKLOAD_CID, WORKLOAD_LIN = 3, 3          # Llama-70B-shaped linear, N=8192, K=28672
 FALLBACK_HBM_GBS = 6650.0
+START_DELAY_CYCLES = 500_000                # ~0.25 ms of SM clock ahead of the start event
 
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
@@ -204,8 +205,6 @@ def run_ours(a, rank: int, world: int, local_rank: int):
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
         sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
         sampler.start()
-    barrier(world)
-    torch.cuda.synchronize(dev)
     if sampler:
         sampler.mark_begin()
     # Clock window: nvidia-smi samples every 100 ms, longer than a short timed
@@ -217,9 +216,15 @@ def run_ours(a, rank: int, world: int, local_rank: int):
         while time.perf_counter() - t_soak < 1.2:
             soak.replay()
             torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):          # graph replays go to the current stream
+        # A device-side delay ahead of the start event: the host has submitted
+        # the timed graphs by the time the stream reaches e0, so the region
+        # measures the launches, not the host's submission latency.
+        torch.cuda._sleep(START_DELAY_CYCLES)
         e0.record(stream)
         for g in graphs:
             g.replay()
@@ -272,7 +277,9 @@ def run_ours(a, rank: int, world: int, local_rank: int):
                    "group_size": 128, "symmetric": sym, "weights": "N(0,0.015) bf16, seeded PCG64",
                    "l2": f"rotating {ncopies} packed-weight copies "
                          f"({ncopies * wbytes / 1e6:.0f} MB > {l2 / 1e6:.0f} MB L2)",
-                   "timing": "CUDA graphs of back-to-back GEMV launches, CUDA events",
+                   "timing": "CUDA graphs of back-to-back GEMV launches, CUDA events; "
+                             "host sync, then a ~0.25 ms device-side delay queued ahead "
+                             "of the start event",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "us_per_linear_per_gpu": round(elapsed_ms * 1e3 / a.steps, 4),
         "hbm_tbs": round(achieved_gbs / 1e3, 4),
@@ -280,7 +287,7 @@ def run_ours(a, rank: int, world: int, local_rank: int):
                      "unit": "GB/s", "frac": round(achieved_gbs / peak, 4), "traffic": traffic,
                      "bytes_per_launch": bytes_per, "peak_source": peak_src,
                      "frac_of_nominal_8tbs": round(achieved_gbs / 8000.0, 4)},
-        "gpu_launches": a.steps,
+        "gpu_launches": 2 * a.steps,          # the streaming GEMV and its split-K finish per step
         "deterministic": deterministic,
         "e2e": e2e,
         "clocks": clocks,
@@ -292,6 +299,9 @@ def run_ours(a, rank: int, world: int, local_rank: int):
         torch.cuda.empty_cache()
         extras["gemm"] = time_gemm(dev, stream)
         extras["layer_awq"] = time_layer_awq(dev, stream)
+        extras["nvfp4"] = time_nvfp4(dev, stream)
+        extras["gptq"] = time_gptq(dev, stream)
+        extras["awq_search"] = time_awq_search(dev, stream)
     line.update(extras)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(W, x, N, K, sym)
@@ -436,8 +446,13 @@ def time_gemm(dev, stream):
         del Wt
         ncopies = max(3, math.ceil(3 * l2 / qw.packed.numel()))
         copies = [qw.packed] + [qw.packed.clone() for _ in range(ncopies - 1)]
-        for M in wl.Ms:
-            x = inputs.workload_activations(cid, li, M)
+        bf16_peak = _measured_bf16_tflops()
+        cases = [(M, 0) for M in wl.Ms] + [(M, 1) for M in wl.Ms]
+        cases += [(M, 0) for M in ((128, 512, 2048) if li == 0 else (512,))]
+        for M, forced in cases:
+            ch = inputs.outlier_channels(K, 0.01, inputs.outlier_seed(cid, K))
+            x = (inputs.workload_activations(cid, li, M) if M <= 64 else
+                 inputs.activations(M, K, seed=M + li, channels=ch, mult=30.0))
             xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
             y = torch.empty((M, N), dtype=torch.float32, device=dev)
             ws_bytes = abi.wq_gemm_workspace_bytes(M, N, K)
@@ -448,8 +463,9 @@ def time_gemm(dev, stream):
                                        ws, ws_bytes, s)
                 assert st == 0
 
-            steps = 1000
-            graphs = build_graphs(launch, stream, steps, 50 * ncopies, dev)
+            steps = 1000 if M <= 64 else (200 if M <= 512 else 40)
+            abi.wq_debug_gemm_force_fold(forced)
+            graphs = build_graphs(launch, stream, steps, min(50 * ncopies, steps), dev)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             with torch.cuda.stream(stream):
@@ -460,11 +476,16 @@ def time_gemm(dev, stream):
                     g.replay()
                 e1.record(stream)
             e1.synchronize()
+            abi.wq_debug_gemm_force_fold(0)
             us = e0.elapsed_time(e1) * 1e3 / steps
             b = algorithmic_bytes(M, N, K, wl.sym)
-            out[f"{N}x{K}_m{M}"] = {"us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1),
-                                    "tflops": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 1),
-                                    "launches": steps + 1}
+            tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            rec = {"us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1),
+                   "tflops": round(tflops, 1), "launches": steps + 1,
+                   "kernel": "many-row (fold)" if (forced or M > 64) else "skinny"}
+            if M > 64 and bf16_peak:
+                rec["tensor_frac_of_measured_bf16"] = round(tflops / bf16_peak, 4)
+            out[f"{N}x{K}_m{M}" + ("_fold" if forced else "")] = rec
         del copies, qw
         torch.cuda.empty_cache()
     if abi.wq_last_device_status(stream) != 0:
@@ -540,6 +561,152 @@ def time_layer_awq(dev, stream):
     del lins
     torch.cuda.empty_cache()
     return out
+
+
+# fp64 rate of a B200 from its unit counts: 148 SMs x 64 fp64 FMA per clock x
+# 2 flops x 1.965 GHz (the calibrated quantizers run on fp64 CUDA cores).
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+# dense FP4 tensor rate: the measured bf16 GEMM rate x 4 (nominal FP4 / bf16)
+FP4_PER_BF16 = 4.0
+
+
+def _events_time(fn, stream, reps, warm=2):
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps          # ms
+
+
+def time_nvfp4(dev, stream):
+    """NVFP4 (W4A4, block-scaled FP4 tensor cores, wq_nvfp4_linear): the
+    8192x28672 down projection at M = 1 and 16 (decode, HBM-bound: 4.5 bits
+    per weight) and the 28672x8192 gate/up projection at M = 128 (a batch of
+    activation rows, reported against the FP4 tensor rate); graphs of
+    back-to-back calls over copies of the packed weight (> L2)."""
+    import numpy as np
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    from post_weight_quantization_wq_b200 import _binding as abi
+    from post_weight_quantization_wq_b200 import inputs
+    out = {}
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    bf16_peak = _measured_bf16_tflops()
+    for (cid, li), Ms in (((3, 3), (1, 16)), ((4, 0), (128,))):
+        W = inputs.workload_weight(cid, li)
+        N, K = W.shape
+        Wt = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+        del W
+        with torch.cuda.stream(stream):
+            qw = wq.nvfp4_quantize(Wt, stream=stream)
+        torch.cuda.synchronize(dev)
+        del Wt
+        ncopies = max(3, math.ceil(3 * l2 / qw.packed.numel()))
+        copies = [qw.packed] + [qw.packed.clone() for _ in range(ncopies - 1)]
+        for M in Ms:
+            x = inputs.activations(M, K, seed=M + 11)
+            xt = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            wsb = abi.wq_nvfp4_linear_workspace_bytes(M, N, K)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+
+            def launch(i, s):
+                st = abi.wq_nvfp4_linear(xt, copies[i % ncopies], qw.tensor_scale, M, N, K, y, ws,
+                                         wsb, s)
+                assert st == 0
+
+            steps = 400
+            graphs = build_graphs(launch, stream, steps, 20 * ncopies, dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                graphs[0].replay()
+                e0.record(stream)
+                for g in graphs:
+                    g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / steps
+            nbytes = N * K // 2 + N * K // 16 + 2 * M * K + 4 * M * N
+            tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            rec = {"us": round(us, 3), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+                   "tflops": round(tflops, 1), "bytes": nbytes}
+            if M >= 128 and bf16_peak:
+                rec["fp4_tensor_frac"] = round(tflops / (bf16_peak * FP4_PER_BF16), 4)
+            out[f"{N}x{K}_m{M}"] = rec
+        del copies, qw
+        torch.cuda.empty_cache()
+    if abi.wq_last_device_status(stream) != 0:
+        raise RuntimeError("device error in the NVFP4 leg")
+    return out
+
+
+def _measured_bf16_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return None
+
+
+def time_gptq(dev, stream, N=4096, K=4096, T=512):
+    """GPTQ on a 4096 x 4096 weight (a Llama-7B attention projection) with 512
+    correlated calibration rows (wq_gptq_quantize: fp64 Hessian, Cholesky,
+    per-group feedback); fp64 flops counted from the algorithm's steps."""
+    import numpy as np
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    from post_weight_quantization_wq_b200 import _binding as abi
+    from post_weight_quantization_wq_b200 import inputs
+    W = torch.from_numpy(inputs.weights(N, K, 0.02, seed=31).view(np.int16)).to(dev).view(torch.bfloat16)
+    X = torch.from_numpy(inputs.correlated_calibration(T, K, seed=32).view(np.int16)).to(dev).view(
+        torch.bfloat16)
+    ws = torch.empty(abi.wq_gptq_workspace_bytes(T, N, K), dtype=torch.uint8, device=dev)
+    ms = _events_time(lambda: wq.gptq_quantize(W, X, workspace=ws, stream=stream), stream, 3, 1)
+    flops = 2.0 * T * K * K + K ** 3 / 3.0 + 2.0 * N * K * K / 2 + (K // 128) * 2.0 * N * 128 * 128
+    return {"shape": f"{N}x{K}", "calib_rows": T, "ms": round(ms, 2),
+            "fp64_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "fp64_peak_tflops_derived": round(FP64_PEAK_TFLOPS, 1)}
+
+
+def time_awq_search(dev, stream):
+    """The AWQ alpha search (21 values) on the decoder layer's q projection
+    (8192 x 8192) with its 128 calibration rows; the loss of each alpha is an
+    fp64 product of the calibration rows with the weight difference."""
+    import numpy as np
+    import torch
+    import post_weight_quantization_wq_b200 as wq
+    from post_weight_quantization_wq_b200 import _binding as abi
+    from post_weight_quantization_wq_b200 import inputs
+    cid, li = 5, 0
+    wl = inputs.WORKLOADS[cid]
+    K = wl.linears[li].K
+    W = inputs.workload_weight(cid, li)
+    N = W.shape[0]
+    X = inputs.activations(wl.calib_rows, K, inputs.calib_seed(cid, K),
+                           inputs.outlier_channels(K, wl.act_outlier_frac, inputs.outlier_seed(cid, K)),
+                           wl.calib_outlier_mult)
+    Wt = torch.from_numpy(W.view(np.int16)).to(dev).view(torch.bfloat16)
+    Xt = torch.from_numpy(X.view(np.int16)).to(dev).view(torch.bfloat16)
+    T = X.shape[0]
+    ws = torch.empty(abi.wq_awq_search_workspace_bytes(T, N, K, 20), dtype=torch.uint8, device=dev)
+    res = {}
+
+    def run():
+        res.update(wq.awq_search(Wt, Xt, workspace=ws, stream=stream))
+    ms = _events_time(run, stream, 2, 1)
+    flops = 21 * 2.0 * T * N * K
+    return {"shape": f"{N}x{K}", "calib_rows": T, "grid": 21, "ms": round(ms, 2),
+            "alpha": res.get("alpha"), "fp64_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "fp64_peak_tflops_derived": round(FP64_PEAK_TFLOPS, 1)}
 
 
 def time_other_m(qw, copies, ncopies, N, K, sym, dev, stream):

@@ -141,9 +141,11 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
 
 /*
  * wq_workspace_bytes -- workspace needed by wq_gemv_w4a16 for M = 1..8
- * (0 when that call needs none), and by wq_gemm_w4a16 for M = 9..64 (the
- * only entry point for those M); 0 for M outside 1..64 or invalid sizes.
- * wq_gemm_workspace_bytes -- workspace needed by wq_gemm_w4a16, M = 1..64.
+ * (0 when that call needs none), and by wq_gemm_w4a16 for M = 9 ..
+ * WQ_GEMM_MAX_M (the only entry point for those M); 0 for other M or invalid
+ * sizes.
+ * wq_gemm_workspace_bytes -- workspace needed by wq_gemm_w4a16,
+ * M = 1..WQ_GEMM_MAX_M.
  * A workspace holds completion counters and split-K partial sums; the GEMM's
  * also holds the per-group sums of x, so every GEMM call needs one.  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
  * the counters: they must be zero before the first call that uses a
@@ -187,16 +189,22 @@ wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* p
                         void* workspace, size_t ws_bytes, wq_stream_t stream);
 
 /*
- * wq_gemm_w4a16 -- the same linear for M = 1..64 activation rows on the
- * tensor cores (tcgen05; the activation tile is zero-padded to 16, 32, 48
- * or 64 rows, so it pays off from about M = 3, where the CUDA-core GEMV
- * becomes issue-bound): per group, the weights are dequantized into tensor
- * memory as bf16 tiles holding the exact integers 128 + q, multiplied with x
- * on the tensor cores with fp32 accumulation, and the group's exact
- * contribution s16 * (D - (128 + z) * sum_k x[m][k]) is added in fp32.  Arguments as wq_gemv_w4a16; inv_act_scale must be NULL
+ * wq_gemm_w4a16 -- the same linear for M = 1..WQ_GEMM_MAX_M activation rows
+ * on the tensor cores (tcgen05).  Per group, the weights are dequantized to
+ * bf16 tiles holding the exact integers 128 + q, multiplied with x on the
+ * tensor cores with fp32 accumulation, and the group's exact contribution
+ * s16 * (D - (128 + z) * sum_k x[m][k]) is added in fp32.  Two kernels:
+ *   - M <= 64 (decode batches; the activation tile zero-padded to 16, 32, 48
+ *     or 64 rows, so it pays off from about M = 3, where the CUDA-core GEMV
+ *     becomes issue-bound): the weights are dequantized into tensor memory;
+ *   - M > 64 (prefill, "大模型量化全景解析", section 八: compute-bound): tiles
+ *     of 128 weight rows x 128 activation rows, the dequantized weights in
+ *     shared memory, the running sums in tensor memory.
+ * Arguments as wq_gemv_w4a16; inv_act_scale must be NULL
  * (WQ_ERR_INVALID_ARG otherwise: the bf16 tensor-core operand cannot hold
  * x * inv_act_scale exactly).
  */
+#define WQ_GEMM_MAX_M 65536
 wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
                         int N, int K, int group_size, int symmetric, int layout, float* y,
                         void* workspace, size_t ws_bytes, wq_stream_t stream);
@@ -373,6 +381,14 @@ wq_status wq_gemv_w4a16_static(const void* x, const float* inv_act_scale, const 
  * calls enqueued afterwards, from any thread.
  */
 void wq_debug_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * wq_debug_gemm_force_fold -- test hook, not part of the stable ABI: 1 makes
+ * wq_gemm_w4a16 use its many-row kernel (M > 64) for every M, so both kernels
+ * can be checked and timed on the same shapes; 0 restores the choice by M.
+ * Affects calls enqueued afterwards, from any thread.
+ */
+void wq_debug_gemm_force_fold(int on);
 
 /*
  * wq_debug_gemv_split -- test hook, not part of the stable ABI: how

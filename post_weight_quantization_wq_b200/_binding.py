@@ -32,6 +32,7 @@ WQ_GPTQ_MAX_T = 65536
 WQ_AWQ_MAX_T = 65536
 WQ_AWQ_MAX_GRID = 1000
 WQ_NVFP4_MAX_M = 128
+WQ_GEMM_MAX_M = 65536
 
 # name -> (restype, argtypes); the exported symbols of include/wq.h
 _P = ctypes.c_void_p
@@ -50,6 +51,7 @@ SIGNATURES = {
     "wq_gemv_w4a16_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "wq_last_device_status": (_I, [_P]),
     "wq_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "wq_debug_gemm_force_fold": (None, [_I]),
     "wq_stream_read_probe": (_I, [_P, _S, _P, _P]),
     "wq_debug_gemv_split": (_I, [_I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "wq_gptq_workspace_bytes": (_S, [_I, _I, _I]),
@@ -171,6 +173,10 @@ def wq_last_device_status(stream=None) -> int:
 
 def wq_debug_set_wait_limit_ns(ns: int) -> None:
     load().wq_debug_set_wait_limit_ns(int(ns))
+
+
+def wq_debug_gemm_force_fold(on: int) -> None:
+    load().wq_debug_gemm_force_fold(int(on))
 
 
 def wq_debug_gemv_split(M, N, K, awq, num_sms, ctas_per_sm):

@@ -19,6 +19,7 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
                         int K, int sym, float* y, void* workspace, int* err, int num_sms,
                         unsigned long long wait_ns, cudaStream_t stream);
 size_t gemm_workspace_bytes(int M, int N, int K);
+void gemm_force_fold(int on);
 size_t gptq_workspace_bytes(int T, int N, int K);
 size_t awq_workspace_bytes(int T, int N, int K, int n_grid);
 cudaError_t launch_nvfp4_quantize(const void* A, int R, int C, uint8_t* codes, uint8_t* scales,
@@ -258,13 +259,13 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
 size_t wq_workspace_bytes(int M, int N, int K) {
   if (N <= 0 || K <= 0 || K % WQ_GROUP_SIZE || N > WQ_MAX_DIM || K > WQ_MAX_DIM) return 0;
   if (M >= 1 && M <= 8) return wq::gemv_workspace_bytes(M, N, K);
-  if (M >= 9 && M <= 64) return wq::gemm_workspace_bytes(M, N, K);
+  if (M >= 9 && M <= WQ_GEMM_MAX_M) return wq::gemm_workspace_bytes(M, N, K);
   return 0;
 }
 
 size_t wq_gemm_workspace_bytes(int M, int N, int K) {
   if (N <= 0 || K <= 0 || K % WQ_GROUP_SIZE || N > WQ_MAX_DIM || K > WQ_MAX_DIM) return 0;
-  if (M < 1 || M > 64) return 0;
+  if (M < 1 || M > WQ_GEMM_MAX_M) return 0;
   return wq::gemm_workspace_bytes(M, N, K);
 }
 
@@ -285,8 +286,8 @@ wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* p
 wq_status wq_gemm_w4a16(const void* x, const float* inv_act_scale, const void* packed, int M,
                         int N, int K, int group_size, int symmetric, int layout, float* y,
                         void* workspace, size_t ws_bytes, wq_stream_t stream) {
-  wq_status st = check_linear(x, inv_act_scale, packed, M, 1, 64, N, K, group_size, symmetric,
-                              layout, y, workspace, ws_bytes, true);
+  wq_status st = check_linear(x, inv_act_scale, packed, M, 1, WQ_GEMM_MAX_M, N, K, group_size,
+                              symmetric, layout, y, workspace, ws_bytes, true);
   if (st != WQ_OK) return st;
   if (inv_act_scale) return WQ_ERR_INVALID_ARG;
   cudaError_t e;
@@ -447,6 +448,11 @@ wq_status wq_last_device_status(wq_stream_t stream) {
 // satisfied give up at once, which exercises the timeout path without
 // stalling the GPU.  Not part of the stable ABI.
 void wq_debug_set_wait_limit_ns(unsigned long long ns) { g_wait_ns.store(ns ? ns : 1ull); }
+
+// Test hook: 1 makes wq_gemm_w4a16 use its many-row kernel for every M (for
+// comparisons at the skinny sizes); 0 restores the choice by M.  Not part of
+// the stable ABI.
+void wq_debug_gemm_force_fold(int on) { wq::gemm_force_fold(on ? 1 : 0); }
 
 // Test hook: how wq_gemv_w4a16 splits its tiles for a given SM count and
 // occupancy (host arithmetic only, no device call).  Not part of the stable ABI.

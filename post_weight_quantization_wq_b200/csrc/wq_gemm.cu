@@ -145,11 +145,6 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, u
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
-__device__ __forceinline__ uint32_t and_or3(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
 
 __device__ __forceinline__ int owner_of(long long u, long long T, int G) {
   return (int)(((u + 1) * G + T - 1) / T) - 1;
@@ -630,10 +625,25 @@ static size_t gemm_partials_bytes(const Geom& g, int M) {
   return g.NS <= 1 ? 0 : (size_t)g.NS * gemm_mpad(M) * g.Npad * sizeof(float);
 }
 
+size_t gemm_fold_workspace_bytes(int M, int N, int K);
+cudaError_t launch_gemm_fold(const void* x, const void* packed, int M, int N, int K, int sym,
+                             float* y, void* workspace, int* err, unsigned long long wait_ns,
+                             cudaStream_t stream);
+
+// Test hook: run the many-row (fold) kernel for every M, so it can be
+// compared with the skinny kernel on the same shapes.
+static int g_force_fold = 0;
+void gemm_force_fold(int on) { g_force_fold = on; }
+
+static bool use_fold(int M) { return M > 64 || g_force_fold; }
+
 size_t gemm_workspace_bytes(int M, int N, int K) {
+  if (M > 64) return gemm_fold_workspace_bytes(M, N, K);
+  const size_t fold = gemm_fold_workspace_bytes(M, N, K);
   const Geom g = make_geom(N, K, 1);
-  return (size_t)kCounterBytes + gemm_partials_bytes(g, M) +
-         (size_t)g.NG * kXsumRow * sizeof(float);
+  const size_t skinny = (size_t)kCounterBytes + gemm_partials_bytes(g, M) +
+                        (size_t)g.NG * kXsumRow * sizeof(float);
+  return skinny > fold ? skinny : fold;
 }
 
 template <int MPAD>
@@ -699,6 +709,8 @@ static cudaError_t launch_gemm_t(const GemmParams& prm, const void* x, int num_s
 cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, int sym,
                         float* y, void* workspace, int* err, int num_sms,
                         unsigned long long wait_ns, cudaStream_t stream) {
+  if (use_fold(M))
+    return launch_gemm_fold(x, packed, M, N, K, sym, y, workspace, err, wait_ns, stream);
   GemmParams prm;
   prm.g = make_geom(N, K, sym);
   prm.packed = static_cast<const uint8_t*>(packed);

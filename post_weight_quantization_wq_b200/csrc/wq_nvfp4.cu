@@ -169,16 +169,19 @@ __global__ void nvfp4_sf_relayout_kernel(const uint8_t* __restrict__ sf, int N, 
 // scales): per 64 inputs one MMA of M = 128 weight rows x N = MPAD activation
 // rows; the block scales of both operands are copied from shared memory into
 // tensor memory (tcgen05.cp) next to the fp32 accumulator; the tensor scales
-// S_w S_x are applied once at the end.  A CTA owns one 128-row tile of W and
-// one contiguous range of K; split-K partial sums are added in a fixed order
-// by a small second kernel.
+// S_w S_x are applied once at the end.  The work is the sequence of (128-row
+// tile of W, 256-input stage) pairs, tile-major; G persistent CTAs each take
+// one contiguous share of it (stream-K), so a CTA ends one tile's piece and
+// starts the next without a new launch, and every SM gets the same number of
+// stages.  The partial sums of the pieces of a tile are added in CTA order by
+// a small second kernel.
 
 struct Fp4GemmParams {
   const uint8_t* w_sf;     // weight scale blocks [ceil(N/128)][K/64][512]
   const uint8_t* x_sf;     // activation scale blocks [K/64][512]
-  float* partials;         // fp32 [KS][MPAD][Npad] raw sums (no tensor scales)
+  float* partials;         // fp32 [tiles][P][MPAD][128] raw sums (no tensor scales)
   int* err;
-  int N, K, M, Npad, KT, KS;
+  int N, K, M, KT, G, P;   // KT stages per tile, G CTAs, P pieces per tile at most
   unsigned long long wait_ns, drain_ns;
 };
 
@@ -194,9 +197,9 @@ struct Fp4Smem {
   static constexpr int kSF = 4 * 512;                   // 4 scale blocks of 64 inputs
   static constexpr int kStage = kA + kB + 2 * kSF;      // multiple of 1024
   static constexpr int kBar = kStages * kStage;
-  static constexpr int kBytes = kBar + (2 * kStages + 1) * 8 + 16;
+  static constexpr int kBytes = kBar + (2 * kStages + 4) * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  static constexpr int kSfCol = 128;                    // scale columns after the accumulator
+  static constexpr int kSfCol = 2 * MPAD;               // scale columns after the 2 accumulators
   static_assert(kSfCol + kStages * 32 <= (int)kFp4TmemCols, "tensor memory");
 };
 
@@ -232,6 +235,10 @@ __device__ __forceinline__ void umma_fp4(uint32_t tmem_d, uint64_t adesc, uint64
       : "memory");
 }
 
+// Persistent: CTA c takes the units (row tile, K split) c, c + grid, ... in
+// order; the TMA ring runs on across units, and the accumulator is double
+// buffered in tensor memory so the epilogue of one unit overlaps the MMAs of
+// the next.
 template <int MPAD>
 __global__ void __launch_bounds__(kFp4Threads, 1)
     nvfp4_gemm_kernel(const Fp4GemmParams p, const __grid_constant__ CUtensorMap wmap,
@@ -243,20 +250,32 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* empty = full + S;
-  uint64_t* accfull = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+  uint64_t* accfull = empty + S;        // [2]
+  uint64_t* accempty = accfull + 2;     // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x, ks = blockIdx.y;
-  const int s0 = (int)((long long)ks * p.KT / p.KS), s1 = (int)((long long)(ks + 1) * p.KT / p.KS);
-  const int nst = s1 - s0;
   const int KB = p.K / 64;                    // scale blocks along K
+  const long long T = (long long)((p.N + 127) / 128) * p.KT;   // stages in all
+  const long long g0 = (long long)blockIdx.x * T / p.G;          // this CTA's share
+  const long long g1 = (long long)(blockIdx.x + 1) * T / p.G;
+  const int b_first = (int)(g0 / p.KT);
+  const int b_end = (int)((g1 - 1) / p.KT) + 1;
+  // stages [s0, s1) of tile b that fall in this CTA's share
+  auto piece = [&](int b, int& s0, int& s1) {
+    const long long lo = (long long)b * p.KT, hi = lo + p.KT;
+    s0 = (int)((g0 > lo ? g0 : lo) - lo);
+    s1 = (int)((g1 < hi ? g1 : hi) - lo);
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(accfull, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accfull[i], 1);
+      mbar_init(&accempty[i], 4);
+    }
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -273,83 +292,107 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    int issued = 0;
+    int i = 0;                              // stages issued by this CTA
     bool ok = true;
-    for (int i = 0; i < nst; ++i) {
-      const int st = i % S;
-      if (i >= S) ok = warp_wait(&empty[st], ((i / S) - 1) & 1, p.wait_ns);
-      if (!ok) break;
-      const int kb0 = 4 * (s0 + i);
-      const int nkb = KB - kb0 < 4 ? KB - kb0 : 4;
-      if (elect_one()) {
-        uint8_t* sa = smem + st * SM::kStage;
-        const uint32_t sfb = (uint32_t)nkb * 512u;
-        mbar_arrive_expect_tx(&full[st], (uint32_t)(SM::kA + SM::kB) + 2u * sfb);
-        tma_load_2d(sa, &wmap, (s0 + i) * 128, b * 128, &full[st]);
-        tma_load_2d(sa + SM::kA, &xmap, (s0 + i) * 128, 0, &full[st]);
-        bulk_copy_g2s(sa + SM::kA + SM::kB, p.w_sf + ((size_t)b * KB + kb0) * 512, sfb, &full[st]);
-        bulk_copy_g2s(sa + SM::kA + SM::kB + SM::kSF, p.x_sf + (size_t)kb0 * 512, sfb, &full[st]);
+    for (int b = b_first; b < b_end && ok; ++b) {
+      int s0, s1;
+      piece(b, s0, s1);
+      for (int sg = s0; sg < s1; ++sg, ++i) {
+        const int st = i % S;
+        if (i >= S) ok = warp_wait(&empty[st], ((i / S) - 1) & 1, p.wait_ns);
+        if (!ok) break;
+        const int kb0 = 4 * sg;
+        const int nkb = KB - kb0 < 4 ? KB - kb0 : 4;
+        if (elect_one()) {
+          uint8_t* sa = smem + st * SM::kStage;
+          const uint32_t sfb = (uint32_t)nkb * 512u;
+          mbar_arrive_expect_tx(&full[st], (uint32_t)(SM::kA + SM::kB) + 2u * sfb);
+          tma_load_2d(sa, &wmap, sg * 128, b * 128, &full[st]);
+          tma_load_2d(sa + SM::kA, &xmap, sg * 128, 0, &full[st]);
+          bulk_copy_g2s(sa + SM::kA + SM::kB, p.w_sf + ((size_t)b * KB + kb0) * 512, sfb,
+                        &full[st]);
+          bulk_copy_g2s(sa + SM::kA + SM::kB + SM::kSF, p.x_sf + (size_t)kb0 * 512, sfb,
+                        &full[st]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      issued = i + 1;
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kDevErrTimeout);
-      for (int k = issued - S < 0 ? 0 : issued - S; k < issued; ++k)
+      for (int k = i - S < 0 ? 0 : i - S; k < i; ++k)
         warp_wait(&full[k % S], (k / S) & 1, p.drain_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = fp4_idesc<MPAD>();
     bool ok = true;
-    int done = 0;
-    for (int i = 0; i < nst; ++i) {
-      const int st = i % S;
-      ok = warp_wait(&full[st], (i / S) & 1, p.wait_ns);
+    int i = 0, lu = 0;
+    for (int b = b_first; b < b_end && ok; ++b, ++lu) {
+      int s0, s1;
+      piece(b, s0, s1);
+      const int db = lu & 1;
+      if (lu >= 2) ok = warp_wait(&accempty[db], ((lu / 2) - 1) & 1, p.wait_ns);
       if (!ok) break;
-      tc_fence_after();
-      const int kb0 = 4 * (s0 + i);
-      const int nkb = KB - kb0 < 4 ? KB - kb0 : 4;
-      if (elect_one()) {
-        const uint32_t sa = smem_u32(smem + st * SM::kStage);
-        const uint32_t tsf = tmem_base + SM::kSfCol + st * 32;
-        for (int kk = 0; kk < nkb; ++kk) {
-          tmem_cp_sf(tsf + kk * 4, sf_block_desc(sa + SM::kA + SM::kB + kk * 512));
-          tmem_cp_sf(tsf + 16 + kk * 4, sf_block_desc(sa + SM::kA + SM::kB + SM::kSF + kk * 512));
+      for (int sg = s0; sg < s1; ++sg, ++i) {
+        const int st = i % S;
+        ok = warp_wait(&full[st], (i / S) & 1, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+        const int kb0 = 4 * sg;
+        const int nkb = KB - kb0 < 4 ? KB - kb0 : 4;
+        if (elect_one()) {
+          const uint32_t sa = smem_u32(smem + st * SM::kStage);
+          const uint32_t tsf = tmem_base + SM::kSfCol + st * 32;
+          for (int kk = 0; kk < nkb; ++kk) {
+            tmem_cp_sf(tsf + kk * 4, sf_block_desc(sa + SM::kA + SM::kB + kk * 512));
+            tmem_cp_sf(tsf + 16 + kk * 4,
+                       sf_block_desc(sa + SM::kA + SM::kB + SM::kSF + kk * 512));
+          }
+          for (int kk = 0; kk < nkb; ++kk)
+            umma_fp4(tmem_base + db * MPAD, umma_desc_sw128(sa + kk * 32),
+                     umma_desc_sw128(sa + SM::kA + kk * 32), idesc,
+                     (sg > s0 || kk > 0) ? 1u : 0u, tsf + kk * 4, tsf + 16 + kk * 4);
+          umma_commit(&empty[st]);
         }
-        for (int kk = 0; kk < nkb; ++kk)
-          umma_fp4(tmem_base, umma_desc_sw128(sa + kk * 32), umma_desc_sw128(sa + SM::kA + kk * 32),
-                   idesc, (i > 0 || kk > 0) ? 1u : 0u, tsf + kk * 4, tsf + 16 + kk * 4);
-        umma_commit(&empty[st]);
+        __syncwarp();
       }
+      if (!ok) break;
+      if (elect_one()) umma_commit(&accfull[db]);
       __syncwarp();
-      done = i + 1;
     }
-    if (ok) {
-      if (elect_one()) umma_commit(accfull);
-      __syncwarp();
-    } else {
+    if (!ok) {
       if (lane == 0) atomicOr(p.err, kDevErrTimeout);
-      if (done > 0) warp_wait(&empty[(done - 1) % S], ((done - 1) / S) & 1, p.drain_ns);
+      if (i > 0) warp_wait(&empty[(i - 1) % S], ((i - 1) / S) & 1, p.drain_ns);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // tensor-memory lane quadrant of this warp
-    const bool ok = nst > 0 && warp_wait(accfull, 0, p.wait_ns);
-    tc_fence_after();
-    if (ok) {
-      const int n = b * 128 + q * 32 + lane;
+    int lu = 0;
+    for (int b = b_first; b < b_end; ++b, ++lu) {
+      const int db = lu & 1;
+      // piece index: this CTA's rank among the CTAs that share tile b
+      const long long s = (long long)b * p.KT;
+      const int c_first = (int)(((s + 1) * p.G - 1) / T);
+      float* out = p.partials +
+                   ((size_t)b * p.P + (size_t)(blockIdx.x - c_first)) * MPAD * 128;
+      if (!warp_wait(&accfull[db], (lu / 2) & 1, p.wait_ns)) {
+        if (lane == 0) atomicOr(p.err, kDevErrTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int nl = q * 32 + lane;
 #pragma unroll
       for (int c = 0; c < MPAD; c += 8) {
         float v[8];
-        tmem_ld8(tmem_base + ((uint32_t)(q * 32) << 16) + c, v);
+        tmem_ld8(tmem_base + ((uint32_t)(q * 32) << 16) + db * MPAD + c, v);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (c + j < p.M) p.partials[((size_t)ks * MPAD + c + j) * p.Npad + n] = v[j];
+          if (c + j < p.M) out[(size_t)(c + j) * 128 + nl] = v[j];
       }
-    } else if (nst > 0 && lane == 0) {
-      atomicOr(p.err, kDevErrTimeout);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[db]);
     }
   }
 
@@ -363,47 +406,57 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
   }
 }
 
-// y[m][n] = (sum over the K splits of the partials, in order) * S_w * S_x.
-__global__ void nvfp4_finish_kernel(const float* __restrict__ partials, int KS, int MPAD, int Npad,
-                                    int M, int N, const float* __restrict__ s_w,
+// y[m][n] = (sum of the pieces of tile n / 128, in CTA order) * S_w * S_x.
+__global__ void nvfp4_finish_kernel(const float* __restrict__ partials, int KT, int G, int P,
+                                    int MPAD, int M, int N, const float* __restrict__ s_w,
                                     const float* __restrict__ s_x, float* __restrict__ y) {
   const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (e >= (long long)M * N) return;
   const int m = (int)(e / N), n = (int)(e % N);
+  const int b = n / 128;
+  const long long T = (long long)((N + 127) / 128) * KT;
+  const long long s_lo = (long long)b * KT, s_hi = s_lo + KT - 1;
+  const int c_first = (int)(((s_lo + 1) * G - 1) / T);
+  const int c_last = (int)(((s_hi + 1) * G - 1) / T);
+  const float* src = partials + ((size_t)b * P * MPAD + m) * 128 + (n & 127);
   float t = 0.0f;
-  for (int k = 0; k < KS; ++k) t += partials[((size_t)k * MPAD + m) * Npad + n];
+  for (int c = 0; c <= c_last - c_first; ++c) t += src[(size_t)c * MPAD * 128];
   y[e] = t * (*s_w * *s_x);
 }
 
 static int fp4_mpad(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 
-// K splits: enough CTAs for the SMs, at least two stages each.
-static int fp4_splits(int NBt, int KT, int num_sms) {
-  int best = 1;
-  double best_eff = 0.0;
-  for (int ks = 1; ks <= 16 && KT / ks >= 2; ++ks) {
-    const long long ctas = (long long)NBt * ks;
-    const long long waves = (ctas + num_sms - 1) / num_sms;
-    const double eff = (double)ctas / (double)(waves * num_sms);
-    if (eff > best_eff + 1e-9 || (ctas < num_sms && ks > best)) {
-      best_eff = eff;
-      best = ks;
-    }
-  }
-  return best;
-}
-
-// The K split is sized for a 148-SM GPU whatever the device, so the workspace
-// size is a function of the shape alone.
+// The stream-K share count G is that of a 148-SM GPU whatever the device, so
+// the workspace size and the order of the final additions are functions of
+// the shape alone (on a smaller GPU the extra CTAs wait for a free SM).
 constexpr int kFp4SplitSms = 148;
+
+struct Fp4Split {
+  int G, P;
+};
+
+// G = min(148, stages); P = the largest number of CTAs whose shares meet one tile.
+static Fp4Split fp4_split(int NBt, int KT) {
+  const long long T = (long long)NBt * KT;
+  Fp4Split sp;
+  sp.G = (int)(T < kFp4SplitSms ? T : kFp4SplitSms);
+  sp.P = 1;
+  for (int b = 0; b < NBt; ++b) {
+    const long long s_lo = (long long)b * KT, s_hi = s_lo + KT - 1;
+    const int c_first = (int)(((s_lo + 1) * sp.G - 1) / T);
+    const int c_last = (int)(((s_hi + 1) * sp.G - 1) / T);
+    if (c_last - c_first + 1 > sp.P) sp.P = c_last - c_first + 1;
+  }
+  return sp;
+}
 
 size_t nvfp4_linear_workspace_bytes(int M, int N, int K) {
   const int NBt = (N + 127) / 128;
   const int KT = (K + kFp4StageK - 1) / kFp4StageK;
-  const int KS = fp4_splits(NBt, KT, kFp4SplitSms);
+  const Fp4Split sp = fp4_split(NBt, KT);
   auto a256 = [](size_t v) { return (v + 255) / 256 * 256; };
   return a256((size_t)M * K / 2) + a256((size_t)(K / 64) * 512) + a256(16) +
-         a256((size_t)KS * fp4_mpad(M) * NBt * 128 * 4);
+         a256((size_t)NBt * sp.P * fp4_mpad(M) * 128 * 4);
 }
 
 template <int MPAD>
@@ -441,8 +494,7 @@ static cudaError_t launch_fp4_gemm(const Fp4GemmParams& prm, const uint8_t* w_co
   if (e != cudaSuccess) return e;
   Fp4GemmParams pp = prm;
   void* args[] = {&pp, &wmap, &xmap};
-  return cudaLaunchKernel(fn, dim3((unsigned)((prm.N + 127) / 128), (unsigned)prm.KS),
-                          dim3(kFp4Threads), args, SM::kAlloc, stream);
+  return cudaLaunchKernel(fn, dim3((unsigned)prm.G), dim3(kFp4Threads), args, SM::kAlloc, stream);
 }
 
 cudaError_t launch_nvfp4_linear(const void* x, const uint8_t* packed, const float* w_scale, int M,
@@ -467,9 +519,10 @@ cudaError_t launch_nvfp4_linear(const void* x, const uint8_t* packed, const floa
   prm.N = N;
   prm.K = K;
   prm.M = M;
-  prm.Npad = NBt * 128;
   prm.KT = KT;
-  prm.KS = fp4_splits(NBt, KT, kFp4SplitSms);
+  const Fp4Split sp = fp4_split(NBt, KT);
+  prm.G = sp.G;
+  prm.P = sp.P;
   prm.wait_ns = wait_ns;
   prm.drain_ns = 1000000000ull;
   switch (fp4_mpad(M)) {
@@ -481,7 +534,7 @@ cudaError_t launch_nvfp4_linear(const void* x, const uint8_t* packed, const floa
   if (e != cudaSuccess) return e;
   const long long outs = (long long)M * N;
   nvfp4_finish_kernel<<<(unsigned)((outs + 255) / 256), 256, 0, stream>>>(
-      partials, prm.KS, fp4_mpad(M), prm.Npad, M, N, w_scale, s_x, y);
+      partials, KT, prm.G, prm.P, fp4_mpad(M), M, N, w_scale, s_x, y);
   return cudaGetLastError();
 }
 

@@ -85,6 +85,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(bar, parity, limit_ns));
 }
 
+// (a & b) | c in one LOP3 with all three operands in registers.
+__device__ __forceinline__ uint32_t and_or3(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // Host: the driver's cuTensorMapEncodeTiled (looked up once), or null.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 

@@ -64,8 +64,12 @@ def test_workspace_bytes():
     assert abi.wq_workspace_bytes(9, 8192, 28672) == gemm16         # M = 9..64: GEMM only
     assert abi.wq_workspace_bytes(64, 8192, 28672) == abi.wq_gemm_workspace_bytes(64, 8192, 28672)
     assert abi.wq_workspace_bytes(0, 8192, 8192) == 0
-    assert abi.wq_workspace_bytes(65, 8192, 8192) == 0
-    assert abi.wq_gemm_workspace_bytes(65, 8192, 8192) == 0
+    # M > 64: the many-row kernel's sums of x [groups][rows padded to 128]
+    # (plus split-K partials when the shape needs them)
+    assert abi.wq_gemm_workspace_bytes(512, 28672, 8192) == C + 64 * 512 * 4
+    assert abi.wq_gemm_workspace_bytes(65, 8192, 8192) >= C + 64 * 128 * 4
+    assert abi.wq_workspace_bytes(65, 8192, 8192) == abi.wq_gemm_workspace_bytes(65, 8192, 8192)
+    assert abi.wq_gemm_workspace_bytes(abi.WQ_GEMM_MAX_M + 1, 8192, 8192) == 0
     assert abi.wq_workspace_bytes(1, 8192, 100) == 0          # K not a multiple of 128
 
 
@@ -91,7 +95,8 @@ def test_quantize_validation_before_launch(args, expect):
 
 
 @pytest.mark.parametrize("fn,M", [("wq_gemv_w4a16", 0), ("wq_gemv_w4a16", 9),
-                                  ("wq_gemm_w4a16", 0), ("wq_gemm_w4a16", 65)])
+                                  ("wq_gemm_w4a16", 0),
+                                  ("wq_gemm_w4a16", abi.WQ_GEMM_MAX_M + 1)])
 def test_linear_rejects_m_out_of_range(fn, M):
     st = getattr(abi, fn)(0x1000, None, 0x2000, M, 256, 1024, 128, 0, 1, 0x3000, 0x4000,
                           1 << 30, 0)
