@@ -147,7 +147,10 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
  * wq_gemm_workspace_bytes -- workspace needed by wq_gemm_w4a16,
  * M = 1..WQ_GEMM_MAX_M.
  * A workspace holds completion counters and split-K partial sums; the GEMM's
- * also holds the per-group sums of x, so every GEMM call needs one.  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
+ * also holds the per-group sums of x, so every GEMM call needs one, and for
+ * the shapes of the GEMV's tensor-core kernel (M = 2..4, K a multiple of 512)
+ * it also holds the activation operand prepared once per 512-input slab, so
+ * every such GEMV call needs one too.  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
  * the counters: they must be zero before the first call that uses a
  * workspace (allocate it zero-filled), and every call that completes leaves
  * them zero again, so one workspace serves any number of later calls of any
@@ -159,23 +162,29 @@ size_t wq_gemm_workspace_bytes(int M, int N, int K);
 
 /*
  * wq_gemv_w4a16 -- the W4A16 decode linear for M = 1..8 activation rows
- * (CUDA cores, dequantization in registers, fp32 accumulation):
+ * (dequantization in registers, fp32 accumulation):
  *
  *   y[m][n] = sum_g s16[n][g] * sum_{k in g} x'[m][k] * (q[n][k] - z[n][g])
  *
- * where x' is the activation as the kernel multiplies it:
- *   - M <= 4 without inv_act_scale (the integer path): each 64-input chunk
- *     of a row of x is rounded to 16-bit fixed point, x' = rn(x * 2^e) * 2^-e
- *     with e chosen so that the chunk's largest |x| lies in [2^14, 2^15)
- *     (that value, and any value with at most 15 - (its exponent gap to the
- *     largest) significant bits, stays exact; every other is within 2^-15 of
- *     the chunk's largest |x|).  The codes times these integers are summed
- *     exactly in int32 (dp4a), so the error in y is at most
- *     2^-15 * sum_k |w_hat[n][k]| * max|x| over k's chunk.  A chunk holding a
- *     NaN or an infinity makes every output of its row NaN.
- *   - otherwise x' = x (bf16, exact in fp32) or, when inv_act_scale is given,
- *     x'[m][k] = fp32(x[m][k]) * inv_act_scale[k] (the AWQ fold,
- *     inv_act_scale = 1/s, one rounded fp32 product).
+ * where x' is the activation as the kernel multiplies it.  Let
+ * u[m][k] = x[m][k] (bf16, exact in fp32), or, when inv_act_scale is given,
+ * u[m][k] = fp32(x[m][k]) * inv_act_scale[k] (the AWQ fold, inv_act_scale =
+ * 1/s, one rounded fp32 product).
+ *   - The integer paths: M = 2..4 with K a multiple of 512 (int8 tensor
+ *     cores, tcgen05.mma kind::i8, with or without inv_act_scale), and
+ *     M <= 4 without inv_act_scale otherwise (CUDA cores, dp4a).  Each
+ *     64-input chunk of a row of u is rounded to 16-bit fixed point,
+ *     x' = rn(u * 2^e) * 2^-e with e chosen so that the chunk's largest |u|
+ *     lies in [2^14, 2^15) (a bf16 value there, and any value with at most
+ *     15 - (its exponent gap to the largest) significant bits, stays exact;
+ *     every other is within 2^-15 of the chunk's largest |u|).  The codes
+ *     times these integers are summed exactly in int32, so the error in y is
+ *     at most 2^-15 * sum_k |w_hat[n][k]| * max|u| over k's chunk.  A chunk
+ *     holding a NaN or an infinity makes every output of its row NaN.  Both
+ *     integer kernels give the same per-chunk integers and differ only in
+ *     the order of the fp32 additions of the chunks' contributions.
+ *   - otherwise (M = 1 with inv_act_scale, M = 5..8, or inv_act_scale with K
+ *     not a multiple of 512) x' = u, multiplied in fp32 on the CUDA cores.
  *   x        bf16 [M][K];      inv_act_scale fp32 [K] or NULL;
  *   packed   the weight in kernel layout `layout` (from wq_pack_layout);
  *   y        fp32 [M][N] out;
@@ -391,12 +400,23 @@ void wq_debug_set_wait_limit_ns(unsigned long long ns);
 void wq_debug_gemm_force_fold(int on);
 
 /*
+ * wq_debug_gemv_force_cuda_cores -- test hook, not part of the stable ABI: 1
+ * makes wq_gemv_w4a16 (and wq_gemv_w4a16_static) use the CUDA-core kernel for
+ * every shape, so it and the tensor-core decode kernel can be checked and
+ * timed on the same shapes; 0 restores the default choice.  Affects calls
+ * enqueued afterwards, from any thread.
+ */
+void wq_debug_gemv_force_cuda_cores(int on);
+
+/*
  * wq_debug_gemv_split -- test hook, not part of the stable ABI: how
  * wq_gemv_w4a16 would split an M x N x K linear (awq != 0: with the
  * activation factor) over a GPU with num_sms SMs holding ctas_per_sm of its
  * CTAs each.  Writes the number of 128 x 512 tiles, the teams per CTA and the
  * CTAs of the grid; team t of the grid's teams T owns tiles
- * [t * tiles / T, (t + 1) * tiles / T).  Host arithmetic only (no device
+ * [t * tiles / T, (t + 1) * tiles / T).  For the shapes of the tensor-core
+ * decode kernel (M = 2..4, K a multiple of 512, not forced onto the CUDA
+ * cores) that is one team per CTA and min(tiles, num_sms) CTAs.  Host arithmetic only (no device
  * call, usable without a GPU).  WQ_ERR_INVALID_ARG for M outside 1..8, N < 1,
  * K not a positive multiple of 128, num_sms or ctas_per_sm < 1, or a null
  * output pointer.

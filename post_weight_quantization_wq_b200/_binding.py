@@ -52,6 +52,7 @@ SIGNATURES = {
     "wq_last_device_status": (_I, [_P]),
     "wq_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "wq_debug_gemm_force_fold": (None, [_I]),
+    "wq_debug_gemv_force_cuda_cores": (None, [_I]),
     "wq_stream_read_probe": (_I, [_P, _S, _P, _P]),
     "wq_debug_gemv_split": (_I, [_I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "wq_gptq_workspace_bytes": (_S, [_I, _I, _I]),
@@ -177,6 +178,10 @@ def wq_debug_set_wait_limit_ns(ns: int) -> None:
 
 def wq_debug_gemm_force_fold(on: int) -> None:
     load().wq_debug_gemm_force_fold(int(on))
+
+
+def wq_debug_gemv_force_cuda_cores(on: int) -> None:
+    load().wq_debug_gemv_force_cuda_cores(int(on))
 
 
 def wq_debug_gemv_split(M, N, K, awq, num_sms, ctas_per_sm):

@@ -20,6 +20,9 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
                         unsigned long long wait_ns, cudaStream_t stream);
 size_t gemm_workspace_bytes(int M, int N, int K);
 void gemm_force_fold(int on);
+void gemv_force_cuda_cores(int on);
+bool gemv_tc_supported(int M, int K);
+bool gemv_forced_cuda_cores();
 size_t gptq_workspace_bytes(int T, int N, int K);
 size_t awq_workspace_bytes(int T, int N, int K, int n_grid);
 cudaError_t launch_nvfp4_quantize(const void* A, int R, int C, uint8_t* codes, uint8_t* scales,
@@ -454,6 +457,8 @@ void wq_debug_set_wait_limit_ns(unsigned long long ns) { g_wait_ns.store(ns ? ns
 // the stable ABI.
 void wq_debug_gemm_force_fold(int on) { wq::gemm_force_fold(on ? 1 : 0); }
 
+void wq_debug_gemv_force_cuda_cores(int on) { wq::gemv_force_cuda_cores(on ? 1 : 0); }
+
 // Test hook: how wq_gemv_w4a16 splits its tiles for a given SM count and
 // occupancy (host arithmetic only, no device call).  Not part of the stable ABI.
 wq_status wq_debug_gemv_split(int M, int N, int K, int awq, int num_sms, int ctas_per_sm,
@@ -462,6 +467,12 @@ wq_status wq_debug_gemv_split(int M, int N, int K, int awq, int num_sms, int cta
       ctas_per_sm < 1 || !tiles || !teams || !grid)
     return WQ_ERR_INVALID_ARG;
   *tiles = wq::gemv_tiles(N, K);
+  if (!wq::gemv_forced_cuda_cores() && wq::gemv_tc_supported(M, K)) {
+    // tensor-core decode kernel: one CTA per SM, one team each
+    *teams = 1;
+    *grid = *tiles < num_sms ? *tiles : num_sms;
+    return WQ_OK;
+  }
   *teams = wq::gemv_teams(M, awq != 0);
   *grid = wq::gemv_grid(*tiles, *teams, num_sms, ctas_per_sm);
   return WQ_OK;

@@ -867,7 +867,43 @@ long long gemv_tiles(int N, int K) {
   return (long long)g.NS * g.NB;
 }
 
+bool gemv_tc_supported(int M, int K);
+cudaError_t launch_gemv_tc(const void* x, const float* inv_s, const void* packed, int M, int N,
+                           int K, int sym, float* y, void* workspace, int* err, int num_sms,
+                           unsigned long long wait_ns, cudaStream_t stream);
+
+// Test hook: route every GEMV to the CUDA-core kernel (0: the tensor-core
+// decode kernel takes the shapes it supports).
+static int g_force_cuda_cores = 0;
+void gemv_force_cuda_cores(int on) { g_force_cuda_cores = on; }
+bool gemv_forced_cuda_cores() { return g_force_cuda_cores != 0; }
+
+// The split-K finish of a persistent GEMV whose G CTAs each own the
+// contiguous run [floor(c T / G), floor((c + 1) T / G)) of the T tiles.
+cudaError_t launch_gemv_finish(const float* partials, float* y, int N, int M, int MP, int NS,
+                               int Npad, int G, long long tiles, cudaStream_t stream) {
+  FinishParams f;
+  f.partials = partials;
+  f.y = y;
+  f.N = N;
+  f.M = M;
+  f.MP = MP;
+  f.NS = NS;
+  f.Npad = Npad;
+  f.G = G;
+  f.tiles = tiles;
+  void* fargs[] = {&f};
+  const long long outs = (long long)M * N;
+  return launch_pdl(reinterpret_cast<const void*>(&gemv_finish_kernel),
+                    dim3((unsigned)((outs + 255) / 256)), dim3(256), fargs, 0, stream);
+}
+
+size_t gemv_tc_workspace_bytes(int M, int N, int K);
+
+// Shapes the tensor-core decode kernel takes get its workspace, which holds
+// the CUDA-core kernel's as a prefix.
 size_t gemv_workspace_bytes(int M, int N, int K) {
+  if (gemv_tc_supported(M, K)) return gemv_tc_workspace_bytes(M, N, K);
   const Geom g = make_geom(N, K, 1);
   if (g.NS <= 1) return 0;
   return (size_t)kCounterBytes + (size_t)g.NS * padded_m(M) * g.Npad * sizeof(float);
@@ -876,6 +912,9 @@ size_t gemv_workspace_bytes(int M, int N, int K) {
 cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, int M, int N,
                         int K, int sym, float* y, void* workspace, int* err, int num_sms,
                         unsigned long long wait_ns, cudaStream_t stream) {
+  if (!g_force_cuda_cores && gemv_tc_supported(M, K))
+    return launch_gemv_tc(x, inv_s, packed, M, N, K, sym, y, workspace, err, num_sms, wait_ns,
+                          stream);
   GemvParams prm;
   prm.g = make_geom(N, K, sym);
   prm.packed = static_cast<const uint8_t*>(packed);
@@ -901,20 +940,8 @@ cudaError_t launch_gemv(const void* x, const float* inv_s, const void* packed, i
   void* args[] = {&prm};
   e = launch_pdl(c.fn, dim3((unsigned)grid), dim3(kGemvThreads * c.teams), args, c.smem, stream);
   if (e != cudaSuccess || prm.g.NS <= 1) return e;
-  FinishParams f;
-  f.partials = prm.partials;
-  f.y = y;
-  f.N = N;
-  f.M = M;
-  f.MP = padded_m(M);
-  f.NS = prm.g.NS;
-  f.Npad = prm.g.Npad;
-  f.G = (int)(grid * c.teams);
-  f.tiles = prm.tiles;
-  void* fargs[] = {&f};
-  const long long outs = (long long)M * N;
-  return launch_pdl(reinterpret_cast<const void*>(&gemv_finish_kernel),
-                    dim3((unsigned)((outs + 255) / 256)), dim3(256), fargs, 0, stream);
+  return launch_gemv_finish(prm.partials, y, N, M, padded_m(M), prm.g.NS, prm.g.Npad,
+                            (int)(grid * c.teams), prm.tiles, stream);
 }
 
 }  // namespace wq

@@ -48,10 +48,33 @@ def test_split_leaves_no_idle_team_inside_a_row_tile(M, awq):
 
 
 def test_split_of_the_headline_linear():
-    """8192 x 28672 at M = 1: 3,584 tiles over one CTA per SM of 148, two
-    teams each (296 teams, 12 or 13 tiles each)."""
+    """8192 x 28672: 3,584 tiles.  At M = 1 (CUDA cores) one CTA per SM of
+    148 with two teams each (296 teams, 12 or 13 tiles each); at M = 2..4 the
+    tensor-core kernel, one team per CTA (24 or 25 tiles each), or two teams
+    again when forced onto the CUDA cores."""
     st, tiles, teams, grid = abi.wq_debug_gemv_split(1, 8192, 28672, 0, 148, 1)
     assert (st, tiles, teams, grid) == (abi.WQ_OK, 3584, 2, 148)
+    for M, awq in ((2, 0), (4, 0), (3, 1)):
+        st, tiles, teams, grid = abi.wq_debug_gemv_split(M, 8192, 28672, awq, 148, 1)
+        assert (st, tiles, teams, grid) == (abi.WQ_OK, 3584, 1, 148)
+    abi.wq_debug_gemv_force_cuda_cores(1)
+    try:
+        st, tiles, teams, grid = abi.wq_debug_gemv_split(2, 8192, 28672, 0, 148, 1)
+    finally:
+        abi.wq_debug_gemv_force_cuda_cores(0)
+    assert (st, tiles, teams, grid) == (abi.WQ_OK, 3584, 2, 148)
+
+
+@pytest.mark.parametrize("forced", [0, 1])
+def test_split_invariants_on_both_kernels(forced):
+    abi.wq_debug_gemv_force_cuda_cores(forced)
+    try:
+        for M in (1, 2, 4):
+            for N, K in ((8192, 28672), (28672, 8192), (128, 28672), (1, 512), (300, 1536)):
+                for sms, per_sm in ((148, 1), (7, 1)):
+                    _check_split(M, N, K, 0, sms, per_sm)
+    finally:
+        abi.wq_debug_gemv_force_cuda_cores(0)
 
 
 @pytest.mark.parametrize("args", [(0, 1, 128, 0, 148, 1), (9, 1, 128, 0, 148, 1),

@@ -1,5 +1,6 @@
-"""The GEMV's integer path (M <= 4, no activation scale) on activations that
-stress its per-chunk 16-bit fixed point: each 64-input chunk of a row of x is
+"""The GEMV's integer paths (M <= 4, no activation scale: the tensor-core
+decode kernel and the CUDA-core kernel, each case on both) on activations that
+stress their per-chunk 16-bit fixed point: each 64-input chunk of a row of x is
 rounded to x_i = rn(x * 2^e) with the chunk's largest |x| in [2^14, 2^15), so
 small values next to large ones in one chunk lose low bits.  The pages
 multiply the dequantized weights with the 16-bit activations themselves
@@ -24,7 +25,8 @@ import post_weight_quantization_wq_b200 as wq
 from post_weight_quantization_wq_b200 import inputs
 from gpu_util import check_close, dev_bf16, quantize_and_check, sample_rows
 
-pytestmark = pytest.mark.gpu
+# every case on both decode kernels (tensor-core and CUDA-core integer paths)
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemv_kernel")]
 
 N_SMALL, K_SMALL = 512, 4096
 
