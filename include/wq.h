@@ -148,7 +148,7 @@ wq_status wq_pack_layout(const uint32_t* qweight, const void* scales, const void
  * M = 1..WQ_GEMM_MAX_M.
  * A workspace holds completion counters and split-K partial sums; the GEMM's
  * also holds the per-group sums of x, so every GEMM call needs one, and for
- * the shapes of the GEMV's tensor-core kernel (M = 2..4, K a multiple of 512)
+ * the shapes of the GEMV's tensor-core kernel (M = 2..8, K a multiple of 512)
  * it also holds the activation operand prepared once per 512-input slab, so
  * every such GEMV call needs one too.  The first WQ_WORKSPACE_COUNTER_BYTES bytes hold
  * the counters: they must be zero before the first call that uses a
@@ -170,7 +170,7 @@ size_t wq_gemm_workspace_bytes(int M, int N, int K);
  * u[m][k] = x[m][k] (bf16, exact in fp32), or, when inv_act_scale is given,
  * u[m][k] = fp32(x[m][k]) * inv_act_scale[k] (the AWQ fold, inv_act_scale =
  * 1/s, one rounded fp32 product).
- *   - The integer paths: M = 2..4 with K a multiple of 512 (int8 tensor
+ *   - The integer paths: M = 2..8 with K a multiple of 512 (int8 tensor
  *     cores, tcgen05.mma kind::i8, with or without inv_act_scale), and
  *     M <= 4 without inv_act_scale otherwise (CUDA cores, dp4a).  Each
  *     64-input chunk of a row of u is rounded to 16-bit fixed point,
@@ -183,8 +183,9 @@ size_t wq_gemm_workspace_bytes(int M, int N, int K);
  *     holding a NaN or an infinity makes every output of its row NaN.  Both
  *     integer kernels give the same per-chunk integers and differ only in
  *     the order of the fp32 additions of the chunks' contributions.
- *   - otherwise (M = 1 with inv_act_scale, M = 5..8, or inv_act_scale with K
- *     not a multiple of 512) x' = u, multiplied in fp32 on the CUDA cores.
+ *   - otherwise (M = 1 with inv_act_scale, or K not a multiple of 512 with
+ *     M = 5..8 or with inv_act_scale) x' = u, multiplied in fp32 on the
+ *     CUDA cores.
  *   x        bf16 [M][K];      inv_act_scale fp32 [K] or NULL;
  *   packed   the weight in kernel layout `layout` (from wq_pack_layout);
  *   y        fp32 [M][N] out;
@@ -415,7 +416,7 @@ void wq_debug_gemv_force_cuda_cores(int on);
  * CTAs each.  Writes the number of 128 x 512 tiles, the teams per CTA and the
  * CTAs of the grid; team t of the grid's teams T owns tiles
  * [t * tiles / T, (t + 1) * tiles / T).  For the shapes of the tensor-core
- * decode kernel (M = 2..4, K a multiple of 512, not forced onto the CUDA
+ * decode kernel (M = 2..8, K a multiple of 512, not forced onto the CUDA
  * cores) that is one team per CTA and min(tiles, num_sms) CTAs.  Host arithmetic only (no device
  * call, usable without a GPU).  WQ_ERR_INVALID_ARG for M outside 1..8, N < 1,
  * K not a positive multiple of 128, num_sms or ctas_per_sm < 1, or a null

@@ -1,4 +1,4 @@
-// wq_gemv_tc.cu -- W4A16 decode linear for M = 2..4 rows of x on the integer
+// wq_gemv_tc.cu -- W4A16 decode linear for M = 2..8 rows of x on the integer
 // tensor cores (tcgen05.mma kind::i8, sm_100a):
 //
 //   y[m][n] = sum_g s16[n][g] * sum_{k in g} x[m][k] * (q[n][k] - z[n][g])
@@ -17,27 +17,22 @@
 // x_i = 256 h + l into signed high bytes h and unsigned low bytes l (the same
 // rounding as the CUDA-core integer path).
 //
-// Weights: the two masks w & 0x0F0F0F0F and w & 0xF0F0F0F0 of a layout word
-// leave its 8 codes in place as unsigned bytes (q for the inputs 0, 4, 1, 5 of
-// the word, 16 q for the inputs 2, 6, 3, 7: nibble slot t holds input 2t for
-// t < 4 and 2(t - 4) + 1 otherwise).  They are the A operand, 128 rows (the
-// tile's output rows) x 512 bytes, stored straight into tensor memory
-// (tcgen05.st) by the unpacking warps: byte 8 j + b of a row is the low mask's
-// byte b (b < 4) or the high mask's byte b - 4 of the row's word j.
+// Weights: w & 0x0F0F0F0F and (w >> 4) & 0x0F0F0F0F of a layout word are its
+// 8 codes as unsigned bytes (the inputs 0, 4, 1, 5 and 2, 6, 3, 7 of the
+// word: nibble slot t holds input 2t for t < 4 and 2(t - 4) + 1 otherwise).
+// They are the A operand, 128 rows (the tile's output rows) x 512 bytes,
+// stored straight into tensor memory (tcgen05.st) by the unpacking warps:
+// bytes 8 j .. 8 j + 7 of a row are those of the row's word j, in that order.
 //
 // B (shared memory, SWIZZLE_128B, K-major, signed bytes, NB = 8, 16 or 32
-// rows for Mpad = 1, 2, 4): for row m of x, rows 4m and 4m + 1 hold h at the
-// byte positions of the low-mask and of the high-mask bytes (zeros
-// elsewhere), rows 4m + 2 and 4m + 3 hold l' = l - 128 likewise; rows 4 Mpad
-// and 4 Mpad + 1 hold ones at the low-mask and at the high-mask positions.
-// Per chunk c (64 bytes of K = two MMAs of K = 32), one accumulator of NB
-// int32 columns:
-//   D[4m] = sum q h,  D[4m+1] = 16 sum q h  (over the two slot classes),
-//   D[4m+2], D[4m+3] likewise with l',  D[4Mp], D[4Mp+1] likewise with 1,
+// rows for Mpad = 2, 4, 8): row 2m holds the high bytes h of row m of x and
+// row 2m + 1 its low bytes as l' = l - 128, both in the input order of the A
+// bytes; row 2 Mpad holds ones.  Per chunk c (64 bytes of K = two MMAs of
+// K = 32), one accumulator of NB int32 columns:
+//   D[2m] = sum q h,  D[2m+1] = sum q l',  D[2Mp] = sum q,
 // so that exactly (l = l' + 128)
-//   sum_{k in c} q x_i = 256 (D[4m] + D[4m+1] / 16) + D[4m+2] + D[4m+3] / 16
-//                        + 128 (D[4Mp] + D[4Mp+1] / 16)
-// (every term fits in int32: 32 products of at most 240 * 128).  The chunk's
+//   sum_{k in c} q x_i = 256 D[2m] + D[2m+1] + 128 D[2Mp]
+// (every term fits in int32: 64 products of at most 15 * 128).  The chunk's
 // contribution to y is then s16 * (that - z * sum_{k in c} x_i) * 2^-e in fp32.
 //
 // The planes depend on the slab of x only, not on the row tile, so a first
@@ -68,7 +63,7 @@
 //               the row tile is shared with another CTA (the small finish
 //               kernel of the CUDA-core path adds the pieces in slab order).
 // Tensor memory (512 columns): four A buffers of 64 columns, then four
-// accumulator sets of 4 NB columns (two at Mpad = 4), one half-tile each.  Every wait is bounded; on timeout the
+// accumulator sets of 4 NB columns (two at Mpad = 8), one half-tile each.  Every wait is bounded; on timeout the
 // kernel records the device error word and winds down, waiting (bounded) for
 // its copies and MMAs in flight.
 #include <cuda.h>
@@ -91,21 +86,21 @@ constexpr int kTgStages = 5;             // code stages (one tile each)
 constexpr int kTgMetaSlots = 4;
 constexpr uint32_t kTgTmemCols = 512;
 constexpr int kTgCodeBytes = kTileRows * kSlabGroups * kCodeBytesPerGroupRow;   // 32 KB
-constexpr int kTgMaxM = 4;
-constexpr int kTgXinfo = kTgMaxM * 8 * 8;           // float2 [4][8 chunks]
+constexpr int kTgMaxM = 8;
+constexpr int kTgXinfo = kTgMaxM * 8 * 8;           // float2 [8][8 chunks]
 constexpr int kTgABufs = 4;              // half-tile A buffers
 constexpr int kTgMeta = kTileRows * kSlabGroups * 4;
 
-// Rows of the B operand (4 per row of x, two rows of ones) and the
+// Rows of the B operand (2 per row of x, one row of ones) and the
 // accumulator sets that fit tensor memory next to the A buffers.
 template <int MP>
 struct TgShape {
-  static constexpr int kNB = MP == 1 ? 8 : MP == 2 ? 16 : 32;     // >= 4 MP + 2
+  static constexpr int kNB = MP == 2 ? 8 : MP == 4 ? 16 : 32;     // >= 2 MP + 1
   static constexpr int kDCols = 4 * kNB;                          // one half-tile
   static constexpr int kDBufs = 256 / kDCols < 4 ? 256 / kDCols : 4;
-  static constexpr int kBSlots = MP == 4 ? 3 : 4;
+  static constexpr int kBSlots = MP == 8 ? 3 : 4;
   static constexpr int kBSlot = kNB * kSlabK;                     // 4 K-blocks x NB rows x 128
-  static constexpr int kRows = 4 * MP;                            // prepared rows per K-block
+  static constexpr int kRows = 2 * MP;                            // prepared rows per K-block
 };
 
 template <int MP>
@@ -131,7 +126,7 @@ constexpr uint32_t kTgColD = 256;        // accumulator sets: columns [256, 512)
 
 struct TgParams {
   const uint8_t* packed;
-  const uint8_t* planes;   // prepared B rows: [NS][4 K-blocks][4 MP rows][128 B]
+  const uint8_t* planes;   // prepared B rows: [NS][4 K-blocks][2 MP rows][128 B]
   const float2* xinfo;     // [NS][MP][8 chunks] (sum x_i, 2^-e)
   float* y;                // fp32 [M][N]
   float* partials;         // fp32 [NS][MP][Npad]
@@ -190,14 +185,14 @@ __device__ __forceinline__ int b_row_chunk(int r, int ck) {
   return r * 128 + (((ck & 7) ^ (r & 7)) << 4);
 }
 
-// Bytes of the prepared rows of one slab: 4 K-blocks x 4 MP rows x 128.
-__host__ __device__ constexpr int tg_slab_plane_bytes(int MP) { return 4 * 4 * MP * 128; }
+// Bytes of the prepared rows of one slab: 4 K-blocks x 2 MP rows x 128.
+__host__ __device__ constexpr int tg_slab_plane_bytes(int MP) { return 4 * 2 * MP * 128; }
 
 // One warp per (slab s, row m < MP of x): the fixed-point bytes of row m of
 // the slab (of x' = x * inv_s when inv_s is given), in the shared-memory
-// order of rows 4m .. 4m + 3 of each K-block, and the chunk factors
+// order of rows 2m and 2m + 1 of each K-block, and the chunk factors
 // (sum x_i, 2^-e).  Rows m >= M are zeros.
-// planes: [NS][4 K-blocks][4 MP rows][128 B]; xinfo: [NS][MP][8].
+// planes: [NS][4 K-blocks][2 MP rows][128 B]; xinfo: [NS][MP][8].
 __global__ void __launch_bounds__(32 * kTgMaxM) gemv_tc_prep_kernel(const uint16_t* __restrict__ x,
                                                                     const float* __restrict__ inv_s,
                                                                     int M, int MP, int K,
@@ -212,11 +207,11 @@ __global__ void __launch_bounds__(32 * kTgMaxM) gemv_tc_prep_kernel(const uint16
   const int c = lane >> 2, sub = lane & 3;   // 64-input chunk and quarter of it
   const int ck = lane;                       // 16-byte chunk of K (words 2 lane, 2 lane + 1)
   const int kb = ck >> 3;                    // K-block of 128 bytes
-  auto row_at = [&](int r) { return ps + kb * 4 * MP * 128 + b_row_chunk(r, ck); };
+  auto row_at = [&](int r) { return ps + kb * 2 * MP * 128 + b_row_chunk(r, ck); };
   if (m >= M) {
     const uint4 z4 = make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) *reinterpret_cast<uint4*>(row_at(4 * m + t)) = z4;
+    *reinterpret_cast<uint4*>(row_at(2 * m)) = z4;
+    *reinterpret_cast<uint4*>(row_at(2 * m + 1)) = z4;
     if (sub == 0) xinfo[((size_t)s * MP + m) * 8 + c] = make_float2(0.0f, 0.0f);
     return;
   }
@@ -275,26 +270,22 @@ __global__ void __launch_bounds__(32 * kTgMaxM) gemv_tc_prep_kernel(const uint16
     xi[q] = bad ? 0 : __float2int_rn(__fmul_rn(__fmul_rn(xf[q], f1), f2));
     sx += xi[q];
   }
-  // bytes of the two words: low-mask positions hold inputs 0, 4, 1, 5,
-  // high-mask positions inputs 2, 6, 3, 7 of each word; l' = l - 128 is the
-  // low byte with its top bit flipped
+  // bytes of the two words in the A byte order: inputs 0, 4, 1, 5, then
+  // 2, 6, 3, 7 of each word; l' = l - 128 is the low byte with its top bit
+  // flipped
   auto hb = [](int a) { return (uint32_t)(a >> 8) & 0xFFu; };
   auto lb = [](int a) { return ((uint32_t)a & 0xFFu) ^ 0x80u; };
-  uint32_t h0[2], h1[2], l0[2], l1[2];
+  uint32_t hw[4], lw[4];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int* v = xi + 8 * t;
-    h0[t] = hb(v[0]) | hb(v[4]) << 8 | hb(v[1]) << 16 | hb(v[5]) << 24;
-    h1[t] = hb(v[2]) | hb(v[6]) << 8 | hb(v[3]) << 16 | hb(v[7]) << 24;
-    l0[t] = lb(v[0]) | lb(v[4]) << 8 | lb(v[1]) << 16 | lb(v[5]) << 24;
-    l1[t] = lb(v[2]) | lb(v[6]) << 8 | lb(v[3]) << 16 | lb(v[7]) << 24;
+    hw[2 * t] = hb(v[0]) | hb(v[4]) << 8 | hb(v[1]) << 16 | hb(v[5]) << 24;
+    hw[2 * t + 1] = hb(v[2]) | hb(v[6]) << 8 | hb(v[3]) << 16 | hb(v[7]) << 24;
+    lw[2 * t] = lb(v[0]) | lb(v[4]) << 8 | lb(v[1]) << 16 | lb(v[5]) << 24;
+    lw[2 * t + 1] = lb(v[2]) | lb(v[6]) << 8 | lb(v[3]) << 16 | lb(v[7]) << 24;
   }
-  // rows 4m, 4m + 2: the low-mask slots of both words; rows 4m + 1, 4m + 3:
-  // the high-mask slots
-  *reinterpret_cast<uint4*>(row_at(4 * m)) = make_uint4(h0[0], 0u, h0[1], 0u);
-  *reinterpret_cast<uint4*>(row_at(4 * m + 1)) = make_uint4(0u, h1[0], 0u, h1[1]);
-  *reinterpret_cast<uint4*>(row_at(4 * m + 2)) = make_uint4(l0[0], 0u, l0[1], 0u);
-  *reinterpret_cast<uint4*>(row_at(4 * m + 3)) = make_uint4(0u, l1[0], 0u, l1[1]);
+  *reinterpret_cast<uint4*>(row_at(2 * m)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *reinterpret_cast<uint4*>(row_at(2 * m + 1)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   sx += __shfl_xor_sync(0xFFFFFFFFu, sx, 1);
   sx += __shfl_xor_sync(0xFFFFFFFFu, sx, 2);
   if (sub == 0) xinfo[((size_t)s * MP + m) * 8 + c] = make_float2((float)sx, unscale);
@@ -359,16 +350,14 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  // Every activation slot once: rows 4 Mpad and 4 Mpad + 1 of each K-block
-  // hold ones at the low-mask and at the high-mask positions, rows past them
-  // zeros; the prepared rows 0 .. 4 Mpad - 1 are copied in per tile.
+  // Every activation slot once: row 2 Mpad of each K-block holds ones, the
+  // rows past it zeros; the prepared rows 0 .. 2 Mpad - 1 are copied in per
+  // tile.
   for (int i = threadIdx.x; i < kBSlots * SH::kBSlot / 16; i += kTgThreads) {
     const int r = (i / 8) % NB;                // 16-byte chunk i: row of its K-block
     const uint32_t one = 0x01010101u;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r == 4 * MP) v = make_uint4(one, 0u, one, 0u);
-    if (r == 4 * MP + 1) v = make_uint4(0u, one, 0u, one);
-    reinterpret_cast<uint4*>(smem + SM::kB)[i] = v;
+    reinterpret_cast<uint4*>(smem + SM::kB)[i] =
+        r == 2 * MP ? make_uint4(one, one, one, one) : make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_shared();            // read by the tensor cores
   if (warp == 1) {
@@ -439,7 +428,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ activations
     // The prepared rows of the tile's slab: for each K-block, rows
-    // 0 .. 4 Mpad - 1 are one contiguous run at the start of its row groups.
+    // 0 .. 2 Mpad - 1 are one contiguous run at the start of its row groups.
     constexpr uint32_t kRun = SH::kRows * 128;
     constexpr uint32_t kBytes = 4 * kRun + MP * 64;
     griddep_wait();                      // the planes come from the preparing kernel
@@ -541,7 +530,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             v[8 * jj + 2 * t] = wd[t] & 0x0F0F0F0Fu;
-            v[8 * jj + 2 * t + 1] = wd[t] & 0xF0F0F0F0u;
+            v[8 * jj + 2 * t + 1] = (wd[t] >> 4) & 0x0F0F0F0Fu;
           }
         }
         tmem_st16(lane_base + jb * 64 + j4 * 16, v);
@@ -595,11 +584,6 @@ __global__ void __launch_bounds__(kTgThreads, 1)
           }
         }
         const float2* xinfo = reinterpret_cast<const float2*>(smem + SM::kXinfo + xs * kTgXinfo);
-        float2 xi[MP][4];
-#pragma unroll
-        for (int m = 0; m < MP; ++m)
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) xi[m][cc] = xinfo[m * 8 + 4 * eh + cc];
         // the four chunks' accumulators, kCS at a time (bounded registers)
         constexpr int kCS = NB >= 32 ? 1 : 2;
         const uint32_t dbase = lane_base + jd * SH::kDCols;
@@ -613,12 +597,12 @@ __global__ void __launch_bounds__(kTgThreads, 1)
           for (int c1 = 0; c1 < kCS; ++c1) {
             const int cc = c2 + c1;
             const int* D = dv[c1];
-            const int ones = 128 * (D[4 * MP] + (D[4 * MP + 1] >> 4));
+            const int ones = 128 * D[2 * MP];
 #pragma unroll
             for (int m = 0; m < MP; ++m) {
-              const int t = 256 * (D[4 * m] + (D[4 * m + 1] >> 4)) + D[4 * m + 2] +
-                            (D[4 * m + 3] >> 4) + ones;
-              run[m] += (sc[cc >> 1] * ((float)t - zc[cc >> 1] * xi[m][cc].x)) * xi[m][cc].y;
+              const float2 xi = xinfo[m * 8 + 4 * eh + cc];   // (sum x_i, 2^-e)
+              const int t = 256 * D[2 * m] + D[2 * m + 1] + ones;
+              run[m] += (sc[cc >> 1] * ((float)t - zc[cc >> 1] * xi.x)) * xi.y;
             }
           }
         }
@@ -700,6 +684,9 @@ cudaError_t launch_tc(const TgParams& prm, int grid, cudaStream_t stream) {
   return launch_pdl(fn, dim3((unsigned)grid), dim3(kTgThreads), args, TgSmem<MP>::kAlloc, stream);
 }
 
+// Rows of x padded to the kernel's instances.
+int tg_mpad(int M) { return M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+
 // Workspace of the tensor-core path: the split-K counters region (unused) and
 // partial sums of the CUDA-core path, then the prepared planes and chunk
 // factors of every slab.
@@ -709,7 +696,7 @@ struct TgWorkspace {
 
 TgWorkspace tg_workspace(int M, int N, int K) {
   const Geom g = make_geom(N, K, 1);
-  const int MP = M <= 2 ? 2 : 4;
+  const int MP = tg_mpad(M);
   auto a256 = [](size_t v) { return (v + 255) / 256 * 256; };
   TgWorkspace w;
   w.partials = kCounterBytes;
@@ -721,7 +708,7 @@ TgWorkspace tg_workspace(int M, int N, int K) {
 
 }  // namespace
 
-// The tensor-core decode path takes M = 2..4 rows of x (with or without the
+// The tensor-core decode path takes M = 2..8 rows of x (with or without the
 // AWQ activation factor) on weights whose every slab is full (K a multiple of
 // 512).  At M = 1 the CUDA-core kernel is faster: each small MMA (N = 8) costs
 // about as much as a large one, so one row of x does not fill the tensor
@@ -744,7 +731,7 @@ cudaError_t launch_gemv_tc(const void* x, const float* inv_s, const void* packed
   prm.partials = reinterpret_cast<float*>(ws + wl.partials);
   prm.err = err;
   prm.M = M;
-  prm.MP = M <= 2 ? 2 : 4;
+  prm.MP = tg_mpad(M);
   prm.tile_rows = kTileRows + kTileRows * prm.g.meta / kCodeBytesPerGroupRow;
   prm.tiles = (long long)prm.g.NS * prm.g.NB;
   prm.wait_ns = wait_ns;
@@ -764,7 +751,8 @@ cudaError_t launch_gemv_tc(const void* x, const float* inv_s, const void* packed
   cudaError_t e;
   switch (prm.MP) {
     case 2: e = launch_tc<2>(prm, grid, stream); break;
-    default: e = launch_tc<4>(prm, grid, stream); break;
+    case 4: e = launch_tc<4>(prm, grid, stream); break;
+    default: e = launch_tc<8>(prm, grid, stream); break;
   }
   if (e != cudaSuccess || prm.g.NS <= 1) return e;
   return launch_gemv_finish(prm.partials, y, N, M, prm.MP, prm.g.NS, prm.g.Npad, grid, prm.tiles,

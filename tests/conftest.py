@@ -30,7 +30,7 @@ def pytest_collection_modifyitems(config, items):
 @pytest.fixture(params=["tensor_cores", "cuda_cores"])
 def gemv_kernel(request):
     """Runs a GEMV test once per decode kernel: the default choice (the
-    integer tensor-core kernel where it applies: M = 2..4, K a multiple of
+    integer tensor-core kernel where it applies: M = 2..8, K a multiple of
     512) and the CUDA-core kernel forced for every shape."""
     from post_weight_quantization_wq_b200 import _binding as abi
     abi.wq_debug_gemv_force_cuda_cores(int(request.param == "cuda_cores"))

@@ -50,20 +50,21 @@ def test_packed_bytes_matches_layout_definition():
 
 def test_workspace_bytes():
     C = abi.WQ_WORKSPACE_COUNTER_BYTES
-    # GEMV, CUDA-core shapes (M = 1, M = 5..8, or K not a multiple of 512):
-    # one slab needs no workspace; otherwise counters + partials
-    # [slabs][padded M][Npad]
+    # GEMV, CUDA-core shapes (M = 1, or K not a multiple of 512): one slab
+    # needs no workspace; otherwise counters + partials [slabs][padded M][Npad]
     assert abi.wq_workspace_bytes(1, 4096, 512) == 0
     assert abi.wq_workspace_bytes(2, 4096, 384) == 0
     assert abi.wq_workspace_bytes(2, 4096, 640) == C + 2 * 2 * 4096 * 4
     assert abi.wq_workspace_bytes(1, 8192, 28672) == C + 56 * 1 * 8192 * 4
-    assert abi.wq_workspace_bytes(5, 8192, 28672) == C + 56 * 8 * 8192 * 4
-    # GEMV, tensor-core shapes (M = 2..4, K a multiple of 512): the same
-    # prefix, then the prepared activation rows per slab (4 K-blocks x 4 Mpad
+    assert abi.wq_workspace_bytes(5, 8192, 28288) == C + 56 * 8 * 8192 * 4
+    # GEMV, tensor-core shapes (M = 2..8, K a multiple of 512): the same
+    # prefix, then the prepared activation rows per slab (4 K-blocks x 2 Mpad
     # rows x 128 B) and the chunk factors (Mpad x 8 float2), each padded to 256 B
-    assert abi.wq_workspace_bytes(2, 4096, 512) == C + 4096 + 256
-    assert abi.wq_workspace_bytes(3, 8192, 28672) == (C + 56 * 4 * 8192 * 4 + 56 * 8192
+    assert abi.wq_workspace_bytes(2, 4096, 512) == C + 2048 + 256
+    assert abi.wq_workspace_bytes(3, 8192, 28672) == (C + 56 * 4 * 8192 * 4 + 56 * 4096
                                                       + 56 * 256)
+    assert abi.wq_workspace_bytes(5, 8192, 28672) == (C + 56 * 8 * 8192 * 4 + 56 * 8192
+                                                      + 56 * 512)
     # GEMM: counters, partials padded to 16-row multiples, sum(x) per group
     gemm16 = C + 56 * 16 * 8192 * 4 + 224 * 64 * 4
     assert abi.wq_gemm_workspace_bytes(1, 4096, 512) == C + 4 * 64 * 4

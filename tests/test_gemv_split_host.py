@@ -49,12 +49,12 @@ def test_split_leaves_no_idle_team_inside_a_row_tile(M, awq):
 
 def test_split_of_the_headline_linear():
     """8192 x 28672: 3,584 tiles.  At M = 1 (CUDA cores) one CTA per SM of
-    148 with two teams each (296 teams, 12 or 13 tiles each); at M = 2..4 the
+    148 with two teams each (296 teams, 12 or 13 tiles each); at M = 2..8 the
     tensor-core kernel, one team per CTA (24 or 25 tiles each), or two teams
     again when forced onto the CUDA cores."""
     st, tiles, teams, grid = abi.wq_debug_gemv_split(1, 8192, 28672, 0, 148, 1)
     assert (st, tiles, teams, grid) == (abi.WQ_OK, 3584, 2, 148)
-    for M, awq in ((2, 0), (4, 0), (3, 1)):
+    for M, awq in ((2, 0), (4, 0), (3, 1), (8, 0), (6, 1)):
         st, tiles, teams, grid = abi.wq_debug_gemv_split(M, 8192, 28672, awq, 148, 1)
         assert (st, tiles, teams, grid) == (abi.WQ_OK, 3584, 1, 148)
     abi.wq_debug_gemv_force_cuda_cores(1)

@@ -131,15 +131,16 @@ def test_workload_full_size(cid, li):
 
 
 @pytest.mark.parametrize("sym", [False, True])
-def test_headline_linear_both_kernels_m1_to_4(sym, gemv_kernel):
+def test_headline_linear_both_kernels(sym, gemv_kernel):
     """8192 x 28672 (the down projection of a Llama-70B-shaped layer) at
-    M = 1..4 on both decode kernels, sampled rows against the oracle."""
+    M = 1, 2, 3, 4, 5, 8 on both decode kernels, sampled rows against the
+    oracle."""
     N, K = 8192, 28672
     W = inputs.weights(N, K, 0.015, seed=123 + sym)
     qw, P, s, z = quantize_and_check(W, None, sym)
     del W
     rows = sample_rows(N, seed=17)
-    for M in (1, 2, 3, 4):
+    for M in (1, 2, 3, 4, 5, 8):
         x = inputs.activations(M, K, seed=40 + M)
         y = wq.linear(dev_bf16(x), qw, path="gemv").cpu().numpy()
         yref = oracle.linear(x, P, s, z, K, sym=sym, rows=rows)

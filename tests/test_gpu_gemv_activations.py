@@ -1,6 +1,7 @@
-"""The GEMV's integer paths (M <= 4, no activation scale: the tensor-core
-decode kernel and the CUDA-core kernel, each case on both) on activations that
-stress their per-chunk 16-bit fixed point: each 64-input chunk of a row of x is
+"""The GEMV's integer paths (the tensor-core decode kernel, M = 2..8, and the
+CUDA-core kernel, M <= 4; each case run on the default choice and with the
+CUDA cores forced) on activations that stress their per-chunk 16-bit fixed
+point: each 64-input chunk of a row of x is
 rounded to x_i = rn(x * 2^e) with the chunk's largest |x| in [2^14, 2^15), so
 small values next to large ones in one chunk lose low bits.  The pages
 multiply the dequantized weights with the 16-bit activations themselves
@@ -45,7 +46,7 @@ def w_small():
 
 
 @pytest.mark.parametrize("mult", [30.0, 50.0])
-@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 6, 8])
 @pytest.mark.parametrize("sym", [False, True])
 def test_outlier_channels(w_small, M, mult, sym):
     ch = inputs.outlier_channels(K_SMALL, 0.01, seed=6)
