@@ -482,7 +482,8 @@ def time_gemm(dev, stream):
             tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
             rec = {"us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1),
                    "tflops": round(tflops, 1), "launches": steps + 1,
-                   "kernel": "many-row (fold)" if (forced or M > 64) else "skinny"}
+                   "kernel": ("many-row (fold)" if (forced or M > 64) else
+                              "int8 decode" if (M <= 16 and K % 512 == 0) else "skinny")}
             if M > 64 and bf16_peak:
                 rec["tensor_frac_of_measured_bf16"] = round(tflops / bf16_peak, 4)
             out[f"{N}x{K}_m{M}" + ("_fold" if forced else "")] = rec

@@ -200,16 +200,20 @@ wq_status wq_gemv_w4a16(const void* x, const float* inv_act_scale, const void* p
 
 /*
  * wq_gemm_w4a16 -- the same linear for M = 1..WQ_GEMM_MAX_M activation rows
- * on the tensor cores (tcgen05).  Per group, the weights are dequantized to
- * bf16 tiles holding the exact integers 128 + q, multiplied with x on the
- * tensor cores with fp32 accumulation, and the group's exact contribution
- * s16 * (D - (128 + z) * sum_k x[m][k]) is added in fp32.  Two kernels:
- *   - M <= 64 (decode batches; the activation tile zero-padded to 16, 32, 48
- *     or 64 rows, so it pays off from about M = 3, where the CUDA-core GEMV
- *     becomes issue-bound): the weights are dequantized into tensor memory;
- *   - M > 64 (prefill, "大模型量化全景解析", section 八: compute-bound): tiles
- *     of 128 weight rows x 128 activation rows, the dequantized weights in
- *     shared memory, the running sums in tensor memory.
+ * on the tensor cores (tcgen05).  Three kernels:
+ *   - M <= 16 with K a multiple of 512 (decode batches): the int8 kernel of
+ *     wq_gemv_w4a16's integer path (codes times the 16-bit fixed-point
+ *     activations of each 64-input chunk, exact int32 sums, same rounding
+ *     and error bound as described there);
+ *   - otherwise M <= 64: per group, the weights are dequantized into tensor
+ *     memory as bf16 tiles holding the exact integers 128 + q, multiplied
+ *     with x (zero-padded to 16, 32, 48 or 64 rows) with fp32 accumulation,
+ *     and the group's exact contribution s16 * (D - (128 + z) * sum_k x[m][k])
+ *     is added in fp32;
+ *   - M > 64 (prefill, "大模型量化全景解析", section 八: compute-bound): the
+ *     same bf16 arithmetic in tiles of 128 weight rows x 128 activation rows,
+ *     the dequantized weights in shared memory, the running sums in tensor
+ *     memory.
  * Arguments as wq_gemv_w4a16; inv_act_scale must be NULL
  * (WQ_ERR_INVALID_ARG otherwise: the bf16 tensor-core operand cannot hold
  * x * inv_act_scale exactly).
@@ -403,9 +407,10 @@ void wq_debug_gemm_force_fold(int on);
 /*
  * wq_debug_gemv_force_cuda_cores -- test hook, not part of the stable ABI: 1
  * makes wq_gemv_w4a16 (and wq_gemv_w4a16_static) use the CUDA-core kernel for
- * every shape, so it and the tensor-core decode kernel can be checked and
- * timed on the same shapes; 0 restores the default choice.  Affects calls
- * enqueued afterwards, from any thread.
+ * every shape, and wq_gemm_w4a16 its bf16 tensor-core kernels, so they and
+ * the int8 tensor-core decode kernel can be checked and timed on the same
+ * shapes; 0 restores the default choice.  Affects calls enqueued afterwards,
+ * from any thread.
  */
 void wq_debug_gemv_force_cuda_cores(int on);
 

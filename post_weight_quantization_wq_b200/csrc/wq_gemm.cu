@@ -637,13 +637,33 @@ void gemm_force_fold(int on) { g_force_fold = on; }
 
 static bool use_fold(int M) { return M > 64 || g_force_fold; }
 
+bool gemm_tc_supported(int M, int K);
+bool gemv_forced_cuda_cores();
+size_t gemv_tc_workspace_bytes(int M, int N, int K);
+cudaError_t launch_gemv_tc(const void* x, const float* inv_s, const void* packed, int M, int N,
+                           int K, int sym, float* y, void* workspace, int* err, int num_sms,
+                           unsigned long long wait_ns, cudaStream_t stream);
+
+// M <= 16 with every slab full goes to the int8 tensor-core decode kernel
+// (unless a test hook forces the bf16 kernels).
+static bool use_int8(int M, int K) {
+  return !g_force_fold && !gemv_forced_cuda_cores() && gemm_tc_supported(M, K);
+}
+
+// Large enough for every kernel the shape may take (the test hooks switch
+// kernels at run time).
 size_t gemm_workspace_bytes(int M, int N, int K) {
   if (M > 64) return gemm_fold_workspace_bytes(M, N, K);
   const size_t fold = gemm_fold_workspace_bytes(M, N, K);
   const Geom g = make_geom(N, K, 1);
   const size_t skinny = (size_t)kCounterBytes + gemm_partials_bytes(g, M) +
                         (size_t)g.NG * kXsumRow * sizeof(float);
-  return skinny > fold ? skinny : fold;
+  size_t need = skinny > fold ? skinny : fold;
+  if (gemm_tc_supported(M, K)) {
+    const size_t tc = gemv_tc_workspace_bytes(M, N, K);
+    if (tc > need) need = tc;
+  }
+  return need;
 }
 
 template <int MPAD>
@@ -709,6 +729,9 @@ static cudaError_t launch_gemm_t(const GemmParams& prm, const void* x, int num_s
 cudaError_t launch_gemm(const void* x, const void* packed, int M, int N, int K, int sym,
                         float* y, void* workspace, int* err, int num_sms,
                         unsigned long long wait_ns, cudaStream_t stream) {
+  if (use_int8(M, K))
+    return launch_gemv_tc(x, nullptr, packed, M, N, K, sym, y, workspace, err, num_sms, wait_ns,
+                          stream);
   if (use_fold(M))
     return launch_gemm_fold(x, packed, M, N, K, sym, y, workspace, err, wait_ns, stream);
   GemmParams prm;

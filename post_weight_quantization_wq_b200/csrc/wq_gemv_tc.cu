@@ -1,5 +1,5 @@
-// wq_gemv_tc.cu -- W4A16 decode linear for M = 2..8 rows of x on the integer
-// tensor cores (tcgen05.mma kind::i8, sm_100a):
+// wq_gemv_tc.cu -- W4A16 decode linear for M = 2..16 rows of x on the
+// integer tensor cores (tcgen05.mma kind::i8, sm_100a):
 //
 //   y[m][n] = sum_g s16[n][g] * sum_{k in g} x[m][k] * (q[n][k] - z[n][g])
 //
@@ -24,8 +24,8 @@
 // stored straight into tensor memory (tcgen05.st) by the unpacking warps:
 // bytes 8 j .. 8 j + 7 of a row are those of the row's word j, in that order.
 //
-// B (shared memory, SWIZZLE_128B, K-major, signed bytes, NB = 8, 16 or 32
-// rows for Mpad = 2, 4, 8): row 2m holds the high bytes h of row m of x and
+// B (shared memory, SWIZZLE_128B, K-major, signed bytes, NB = 8, 16, 32 or
+// 48 rows for Mpad = 2, 4, 8, 16): row 2m holds the high bytes h of row m of x and
 // row 2m + 1 its low bytes as l' = l - 128, both in the input order of the A
 // bytes; row 2 Mpad holds ones.  Per chunk c (64 bytes of K = two MMAs of
 // K = 32), one accumulator of NB int32 columns:
@@ -62,8 +62,9 @@
 //               tile, which is written to y, or to the split-K workspace when
 //               the row tile is shared with another CTA (the small finish
 //               kernel of the CUDA-core path adds the pieces in slab order).
-// Tensor memory (512 columns): four A buffers of 64 columns, then four
-// accumulator sets of 4 NB columns (two at Mpad = 8), one half-tile each.  Every wait is bounded; on timeout the
+// Tensor memory (512 columns): four A buffers of 64 columns (two at
+// Mpad = 16), then up to four accumulator sets of 4 NB columns (two at
+// Mpad = 8 and 16), one half-tile each.  Every wait is bounded; on timeout the
 // kernel records the device error word and winds down, waiting (bounded) for
 // its copies and MMAs in flight.
 #include <cuda.h>
@@ -82,47 +83,49 @@ namespace {
 
 constexpr int kTgWarps = 20;
 constexpr int kTgThreads = kTgWarps * 32;
-constexpr int kTgStages = 5;             // code stages (one tile each)
 constexpr int kTgMetaSlots = 4;
 constexpr uint32_t kTgTmemCols = 512;
 constexpr int kTgCodeBytes = kTileRows * kSlabGroups * kCodeBytesPerGroupRow;   // 32 KB
-constexpr int kTgMaxM = 8;
-constexpr int kTgXinfo = kTgMaxM * 8 * 8;           // float2 [8][8 chunks]
-constexpr int kTgABufs = 4;              // half-tile A buffers
+constexpr int kTgMaxM = 16;
 constexpr int kTgMeta = kTileRows * kSlabGroups * 4;
 
-// Rows of the B operand (2 per row of x, one row of ones) and the
-// accumulator sets that fit tensor memory next to the A buffers.
+// Rows of the B operand (2 per row of x, one row of ones), the tensor-memory
+// split between A buffers (64 columns each) and accumulator sets (one
+// half-tile each), and the shared-memory rings.
 template <int MP>
 struct TgShape {
-  static constexpr int kNB = MP == 2 ? 8 : MP == 4 ? 16 : 32;     // >= 2 MP + 1
-  static constexpr int kDCols = 4 * kNB;                          // one half-tile
-  static constexpr int kDBufs = 256 / kDCols < 4 ? 256 / kDCols : 4;
-  static constexpr int kBSlots = MP == 8 ? 3 : 4;
+  static constexpr int kNB = MP == 2 ? 8 : MP == 4 ? 16 : MP == 8 ? 32 : 48;   // >= 2 MP + 1
+  static constexpr int kDCols = 4 * kNB;
+  static constexpr int kABufs = MP == 16 ? 2 : 4;
+  static constexpr int kColD = kABufs * 64;
+  static constexpr int kDFit = (512 - kColD) / kDCols;
+  static constexpr int kDBufs = kDFit < 4 ? kDFit : 4;
+  static constexpr int kStages = MP == 16 ? 4 : 5;                // code stages (one tile each)
+  static constexpr int kBSlots = MP == 16 ? 2 : MP == 8 ? 3 : 4;
   static constexpr int kBSlot = kNB * kSlabK;                     // 4 K-blocks x NB rows x 128
   static constexpr int kRows = 2 * MP;                            // prepared rows per K-block
+  static constexpr int kXinfo = MP * 8 * 8;                       // float2 [MP][8 chunks]
+  static_assert(kDBufs >= 2 && kColD + kDBufs * kDCols <= 512, "tensor memory");
 };
 
 template <int MP>
 struct TgSmem {
   using SH = TgShape<MP>;
   static constexpr int kCode = 0;
-  static constexpr int kB = kCode + kTgStages * kTgCodeBytes;
+  static constexpr int kB = kCode + SH::kStages * kTgCodeBytes;
   static constexpr int kMeta = kB + SH::kBSlots * SH::kBSlot;
   static constexpr int kXinfo = kMeta + kTgMetaSlots * kTgMeta;
-  static constexpr int kExch = kXinfo + SH::kBSlots * kTgXinfo;       // float [4][32][4]
-  static constexpr int kBar = kExch + 4 * 32 * kTgMaxM * 4;
+  static constexpr int kExch = kXinfo + SH::kBSlots * SH::kXinfo;    // float [4][32][MP]
+  static constexpr int kBar = kExch + 4 * 32 * MP * 4;
   // cfull/cempty, mfull/mempty, bfull/bempty/xiempty, afull/aempty, dfull/dempty
-  static constexpr int kNumBars = 2 * kTgStages + 2 * kTgMetaSlots + 3 * SH::kBSlots +
-                                  2 * kTgABufs + 2 * SH::kDBufs;
+  static constexpr int kNumBars = 2 * SH::kStages + 2 * kTgMetaSlots + 3 * SH::kBSlots +
+                                  2 * SH::kABufs + 2 * SH::kDBufs;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kB % 1024 == 0 && kBar % 8 == 0, "alignment");
   static_assert(kAlloc <= 232448, "shared memory");
 };
 
-constexpr uint32_t kTgColA = 0;          // A buffers: columns [0, 256)
-constexpr uint32_t kTgColD = 256;        // accumulator sets: columns [256, 512)
 
 struct TgParams {
   const uint8_t* packed;
@@ -155,12 +158,13 @@ __device__ __forceinline__ void umma_i8_ts(uint32_t tmem_d, uint32_t tmem_a, uin
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
-// N consecutive 32-bit columns of this thread's lane (N = 8, 16 or 32).
+// N consecutive 32-bit columns of this thread's lane (N a multiple of 8).
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, int* v) {
-  if constexpr (N == 32) {
+  static_assert(N % 8 == 0, "columns");
+  if constexpr (N > 16) {
     tmem_ld_cols<16>(taddr, v);
-    tmem_ld_cols<16>(taddr + 16, v + 16);
+    tmem_ld_cols<N - 16>(taddr + 16, v + 16);
   } else if constexpr (N == 16) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -297,6 +301,8 @@ __global__ void __launch_bounds__(kTgThreads, 1)
   using SH = TgShape<MP>;
   using SM = TgSmem<MP>;
   constexpr int NB = SH::kNB, kBSlots = SH::kBSlots, kDBufs = SH::kDBufs;
+  constexpr int kTgStages = SH::kStages, kTgABufs = SH::kABufs;
+  constexpr uint32_t kTgColA = 0, kTgColD = SH::kColD;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -447,7 +453,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
         mbar_arrive_expect_tx(&bfull[xs], kBytes);
         for (int kb = 0; kb < 4; ++kb)
           bulk_copy_g2s(bslot + kb * (NB / 8) * 1024, src + kb * kRun, kRun, &bfull[xs]);
-        bulk_copy_g2s(smem + SM::kXinfo + xs * kTgXinfo, prm.xinfo + (size_t)s * MP * 8,
+        bulk_copy_g2s(smem + SM::kXinfo + xs * SH::kXinfo, prm.xinfo + (size_t)s * MP * 8,
                       MP * 64, &bfull[xs]);
       }
       __syncwarp();
@@ -547,7 +553,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
     const int eh = (warp - 12) >> 2;           // half-tile: chunks 4 eh .. 4 eh + 3 (groups 2 eh, 2 eh + 1)
     const int r = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + ((uint32_t)(quad * 32) << 16) + kTgColD;
-    float* exch = reinterpret_cast<float*>(smem + SM::kExch) + (quad * 32 + lane) * kTgMaxM;
+    float* exch = reinterpret_cast<float*>(smem + SM::kExch) + (quad * 32 + lane) * MP;
     float run[MP];
 #pragma unroll
     for (int m = 0; m < MP; ++m) run[m] = 0.0f;
@@ -583,7 +589,7 @@ __global__ void __launch_bounds__(kTgThreads, 1)
             zc[gg] = __high2float(sz);
           }
         }
-        const float2* xinfo = reinterpret_cast<const float2*>(smem + SM::kXinfo + xs * kTgXinfo);
+        const float2* xinfo = reinterpret_cast<const float2*>(smem + SM::kXinfo + xs * SH::kXinfo);
         // the four chunks' accumulators, kCS at a time (bounded registers)
         constexpr int kCS = NB >= 32 ? 1 : 2;
         const uint32_t dbase = lane_base + jd * SH::kDCols;
@@ -685,7 +691,7 @@ cudaError_t launch_tc(const TgParams& prm, int grid, cudaStream_t stream) {
 }
 
 // Rows of x padded to the kernel's instances.
-int tg_mpad(int M) { return M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+int tg_mpad(int M) { return M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
 
 // Workspace of the tensor-core path: the split-K counters region (unused) and
 // partial sums of the CUDA-core path, then the prepared planes and chunk
@@ -713,7 +719,10 @@ TgWorkspace tg_workspace(int M, int N, int K) {
 // 512).  At M = 1 the CUDA-core kernel is faster: each small MMA (N = 8) costs
 // about as much as a large one, so one row of x does not fill the tensor
 // cores.
-bool gemv_tc_supported(int M, int K) { return M >= 2 && M <= kTgMaxM && K % kSlabK == 0; }
+bool gemv_tc_supported(int M, int K) { return M >= 2 && M <= 8 && K % kSlabK == 0; }
+
+// The same kernel serves the tensor-core GEMM entry for M = 1..16.
+bool gemm_tc_supported(int M, int K) { return M >= 1 && M <= kTgMaxM && K % kSlabK == 0; }
 
 size_t gemv_tc_workspace_bytes(int M, int N, int K) { return tg_workspace(M, N, K).total; }
 
@@ -745,14 +754,15 @@ cudaError_t launch_gemv_tc(const void* x, const float* inv_s, const void* packed
     int Mv = M, MPv = prm.MP, Kv = K;
     void* args[] = {&xp, &inv_s, &Mv, &MPv, &Kv, &planes, &xinfo};
     cudaError_t e = launch_pdl(reinterpret_cast<const void*>(&gemv_tc_prep_kernel),
-                               dim3((unsigned)prm.g.NS), dim3(32 * kTgMaxM), args, 0, stream);
+                               dim3((unsigned)prm.g.NS), dim3(32 * prm.MP), args, 0, stream);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e;
   switch (prm.MP) {
     case 2: e = launch_tc<2>(prm, grid, stream); break;
     case 4: e = launch_tc<4>(prm, grid, stream); break;
-    default: e = launch_tc<8>(prm, grid, stream); break;
+    case 8: e = launch_tc<8>(prm, grid, stream); break;
+    default: e = launch_tc<16>(prm, grid, stream); break;
   }
   if (e != cudaSuccess || prm.g.NS <= 1) return e;
   return launch_gemv_finish(prm.partials, y, N, M, prm.MP, prm.g.NS, prm.g.Npad, grid, prm.tiles,

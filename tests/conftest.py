@@ -27,13 +27,14 @@ def pytest_collection_modifyitems(config, items):
             item.add_marker(skip)
 
 
-@pytest.fixture(params=["tensor_cores", "cuda_cores"])
-def gemv_kernel(request):
-    """Runs a GEMV test once per decode kernel: the default choice (the
-    integer tensor-core kernel where it applies: M = 2..8, K a multiple of
-    512) and the CUDA-core kernel forced for every shape."""
+@pytest.fixture(params=["int8_tc", "int8_off"])
+def decode_kernel(request):
+    """Runs a linear test once per decode kernel: the default choice (the
+    int8 tensor-core kernel where it applies: wq_gemv_w4a16 at M = 2..8 and
+    wq_gemm_w4a16 at M <= 16, K a multiple of 512) and with that kernel
+    switched off (the CUDA-core GEMV, the bf16 tensor-core GEMM)."""
     from post_weight_quantization_wq_b200 import _binding as abi
-    abi.wq_debug_gemv_force_cuda_cores(int(request.param == "cuda_cores"))
+    abi.wq_debug_gemv_force_cuda_cores(int(request.param == "int8_off"))
     try:
         yield request.param
     finally:

@@ -66,12 +66,17 @@ def test_workspace_bytes():
     assert abi.wq_workspace_bytes(5, 8192, 28672) == (C + 56 * 8 * 8192 * 4 + 56 * 8192
                                                       + 56 * 512)
     # GEMM: counters, partials padded to 16-row multiples, sum(x) per group
+    # (M <= 16 with K a multiple of 512: the largest of that and the int8
+    # kernel's, whose prepared rows take 4 x 2 Mpad x 128 B and chunk
+    # factors Mpad x 64 B per slab)
     gemm16 = C + 56 * 16 * 8192 * 4 + 224 * 64 * 4
-    assert abi.wq_gemm_workspace_bytes(1, 4096, 512) == C + 4 * 64 * 4
+    tc16 = C + 56 * 16 * 8192 * 4 + 56 * 16384 + 56 * 1024
+    assert abi.wq_gemm_workspace_bytes(1, 4096, 512) == C + 2048 + 256
+    assert abi.wq_gemm_workspace_bytes(1, 4096, 1408) == C + 3 * 16 * 4096 * 4 + 11 * 64 * 4
     assert abi.wq_gemm_workspace_bytes(1, 8192, 28672) == gemm16
-    assert abi.wq_gemm_workspace_bytes(16, 8192, 28672) == gemm16
+    assert abi.wq_gemm_workspace_bytes(16, 8192, 28672) == tc16
     assert abi.wq_gemm_workspace_bytes(17, 8192, 28672) == C + 56 * 32 * 8192 * 4 + 224 * 64 * 4
-    assert abi.wq_workspace_bytes(9, 8192, 28672) == gemm16         # M = 9..64: GEMM only
+    assert abi.wq_workspace_bytes(9, 8192, 28672) == tc16           # M = 9..64: GEMM only
     assert abi.wq_workspace_bytes(64, 8192, 28672) == abi.wq_gemm_workspace_bytes(64, 8192, 28672)
     assert abi.wq_workspace_bytes(0, 8192, 8192) == 0
     # M > 64: the many-row kernel's sums of x [groups][rows padded to 128]

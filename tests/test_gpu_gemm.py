@@ -1,5 +1,7 @@
-"""GPU W4A16 skinny GEMM (M = 1..64, tcgen05 tensor cores) against the CPU
-oracle's fp64 linear: rel-L2 <= 1e-3 and max-abs <= 1e-2 * rms(y)."""
+"""GPU W4A16 GEMM entry at M = 1..64 (tcgen05 tensor cores: the int8 decode
+kernel at M <= 16 with K a multiple of 512, the bf16 skinny kernel otherwise;
+the M <= 16 cases run on both) against the CPU oracle's fp64 linear:
+rel-L2 <= 1e-3 and max-abs <= 1e-2 * rms(y)."""
 import numpy as np
 import pytest
 
@@ -12,8 +14,9 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("sym", [False, True])
-@pytest.mark.parametrize("N,K", [(128, 128), (200, 640), (256, 1024), (384, 2048), (129, 11008)])
-def test_gemm_small(N, K, sym):
+@pytest.mark.parametrize("N,K", [(128, 128), (200, 640), (256, 1024), (384, 2048), (129, 11008),
+                                 (300, 1536)])
+def test_gemm_small(N, K, sym, decode_kernel):
     W = inputs.weights(N, K, 0.02, seed=3 * N + K)
     qw, P, s, z = quantize_and_check(W, None, sym)
     for M in (1, 3, 8, 16, 24, 32, 40, 48, 64):
@@ -35,7 +38,7 @@ def test_gemm_zero_point_outside_code_range():
     check_close(y, oracle.linear(x, P, s, z, K, sym=False))
 
 
-def test_gemm_row_tile_split_across_many_ctas():
+def test_gemm_row_tile_split_across_many_ctas(decode_kernel):
     N, K = 128, 28672
     W = inputs.weights(N, K, 0.015, seed=21)
     qw, P, s, z = quantize_and_check(W, None, False)
@@ -54,7 +57,7 @@ def test_gemm_deterministic():
 
 
 @pytest.mark.parametrize("li", [0, 1])
-def test_workload_batched_decode_full_size(li):
+def test_workload_batched_decode_full_size(li, decode_kernel):
     """The batched-decode workload at full size (28672x8192 and 8192x28672,
     M = 16, 32, 64, 1% activation channels x30), sampled output rows."""
     cid = 4

@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("sym", [False, True])
 @pytest.mark.parametrize("N,K", [(1, 128), (200, 640), (256, 1024), (130, 1408), (384, 2048),
                                  (129, 11008), (1, 512), (200, 1536), (129, 5120)])
-def test_gemv_small_all_m(N, K, sym, gemv_kernel):
+def test_gemv_small_all_m(N, K, sym, decode_kernel):
     W = inputs.weights(N, K, 0.02, seed=N + K)
     qw, P, s, z = quantize_and_check(W, None, sym)
     for M in range(1, 9):
@@ -25,7 +25,7 @@ def test_gemv_small_all_m(N, K, sym, gemv_kernel):
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4])
-def test_gemv_row_tile_split_across_many_ctas(M, gemv_kernel):
+def test_gemv_row_tile_split_across_many_ctas(M, decode_kernel):
     """N = 128 with K = 28672: one row tile of 56 slabs, more CTAs than a row
     tile has slabs, so every CTA holds a piece and the last one adds them."""
     N, K = 128, 28672
@@ -37,7 +37,7 @@ def test_gemv_row_tile_split_across_many_ctas(M, gemv_kernel):
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 8])
-def test_gemv_awq_fold_small(M, gemv_kernel):
+def test_gemv_awq_fold_small(M, decode_kernel):
     N, K = 256, 1536
     W = inputs.weights(N, K, 0.015, seed=91)
     chans = inputs.outlier_channels(K, 0.01, seed=92)
@@ -51,7 +51,7 @@ def test_gemv_awq_fold_small(M, gemv_kernel):
     check_close(y, yref, f"awq M={M}")
 
 
-def test_gemv_nonfinite_group_gives_nan_rows(gemv_kernel):
+def test_gemv_nonfinite_group_gives_nan_rows(decode_kernel):
     N, K = 64, 1024
     w = (np.random.default_rng(1).standard_normal((N, K)) * 0.02).astype(np.float32)
     w[9, 300] = np.inf
@@ -65,7 +65,7 @@ def test_gemv_nonfinite_group_gives_nan_rows(gemv_kernel):
     check_close(y[:, keep], yref[:, keep])
 
 
-def test_gemv_deterministic_and_workspace_reuse(gemv_kernel):
+def test_gemv_deterministic_and_workspace_reuse(decode_kernel):
     """Bit-identical reruns; one workspace shared by calls of different sizes
     (the completion counters are left at zero by every call)."""
     import torch
@@ -86,7 +86,7 @@ def test_gemv_deterministic_and_workspace_reuse(gemv_kernel):
 
 
 @pytest.mark.parametrize("N,K", [(1, 2048), (64, 1664), (100, 3200), (128, 3584), (600, 1024)])
-def test_gemv_small_grid_finishes_every_row_tile(N, K, gemv_kernel):
+def test_gemv_small_grid_finishes_every_row_tile(N, K, decode_kernel):
     """Tile counts one more than a multiple of three at M = 1 (three teams per
     CTA): a grid with two teams more than tiles would leave a team without
     tiles among a row tile's owners, and that row tile's split-K sum would
@@ -131,7 +131,7 @@ def test_workload_full_size(cid, li):
 
 
 @pytest.mark.parametrize("sym", [False, True])
-def test_headline_linear_both_kernels(sym, gemv_kernel):
+def test_headline_linear_both_kernels(sym, decode_kernel):
     """8192 x 28672 (the down projection of a Llama-70B-shaped layer) at
     M = 1, 2, 3, 4, 5, 8 on both decode kernels, sampled rows against the
     oracle."""
@@ -144,4 +144,4 @@ def test_headline_linear_both_kernels(sym, gemv_kernel):
         x = inputs.activations(M, K, seed=40 + M)
         y = wq.linear(dev_bf16(x), qw, path="gemv").cpu().numpy()
         yref = oracle.linear(x, P, s, z, K, sym=sym, rows=rows)
-        check_close(y[:, rows], yref, f"{gemv_kernel} sym={sym} M={M}")
+        check_close(y[:, rows], yref, f"{decode_kernel} sym={sym} M={M}")

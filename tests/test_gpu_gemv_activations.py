@@ -27,7 +27,7 @@ from post_weight_quantization_wq_b200 import inputs
 from gpu_util import check_close, dev_bf16, quantize_and_check, sample_rows
 
 # every case on both decode kernels (tensor-core and CUDA-core integer paths)
-pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemv_kernel")]
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("decode_kernel")]
 
 N_SMALL, K_SMALL = 512, 4096
 

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 DEFAULT_WAIT_NS = 2_000_000_000
 
 
-@pytest.mark.parametrize("M,path", [(1, "gemv"), (16, "gemm")])
+@pytest.mark.parametrize("M,path", [(1, "gemv"), (4, "gemv"), (16, "gemm"), (24, "gemm")])
 def test_wait_timeout_is_reported_and_context_stays_usable(M, path):
     import torch
     N, K = 4096, 8192
@@ -43,7 +43,7 @@ def test_wait_timeout_is_reported_and_context_stays_usable(M, path):
     check_close(y, oracle.linear(x, P, s, z, K, sym=False), f"{path} after a timeout")
 
 
-@pytest.mark.parametrize("M,path", [(1, "gemv"), (16, "gemm")])
+@pytest.mark.parametrize("M,path", [(1, "gemv"), (4, "gemv"), (16, "gemm"), (24, "gemm")])
 def test_timeout_with_the_cached_workspace(M, path):
     """linear() without a workspace uses one cached per (device, stream).  A
     call cut short by a timeout may leave its completion counters set;
