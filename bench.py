@@ -44,8 +44,8 @@ START_DELAY_CYCLES = 500_000                # ~0.25 ms of SM clock ahead of the 
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": "dc88ca99b2c212b1f9f775a86df303feb326e54421843fe9827b0f7b53035210",
-               "bytes_per_launch": 124916736 + 3988992}
+NCU_TRAFFIC = {"sources_sha256": "f6bcea9a68a9755c59f6f0ce9a43eb4ab085cd41fd47e75320abd780503f3766",
+               "bytes_per_launch": 124886016 + 3194624}
 
 
 def _args():
@@ -56,7 +56,7 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the offline and other-M legs")
-    ap.add_argument("--case", choices=["gemv_m1", "gemm_m16", "gemm_m64"], default=None,
+    ap.add_argument("--case", choices=["gemv_m1", "gemv_m4", "gemm_m16", "gemm_m64"], default=None,
                     help="run one small profiling case (3 launches) and exit")
     return ap.parse_args()
 
@@ -906,24 +906,29 @@ def max_over_ranks(v, world, dev):
 
 
 def run_case(a):
-    """A few launches of one kernel on one workload, for profilers: gemv_m1 =
-    wq_gemv_w4a16 on 8192x28672 at M = 1; gemm_m16 / gemm_m64 = wq_gemm_w4a16
-    on 28672x8192 at M = 16 / 64 (asymmetric).  About 1 GB on the device."""
+    """A few launches of one kernel on one workload, for profilers: gemv_m1 /
+    gemv_m4 = wq_gemv_w4a16 on 8192x28672 at M = 1 (CUDA cores) / 4 (int8
+    tensor cores); gemm_m16 / gemm_m64 = wq_gemm_w4a16 on 28672x8192 at
+    M = 16 (int8 tensor cores) / 64 (bf16 tensor cores), asymmetric.  About
+    1 GB on the device."""
     import numpy as np
     import torch
     import post_weight_quantization_wq_b200 as wq
     from post_weight_quantization_wq_b200 import inputs
-    cid, li, M = {"gemv_m1": (WORKLOAD_CID, WORKLOAD_LIN, 1), "gemm_m16": (4, 0, 16),
+    cid, li, M = {"gemv_m1": (WORKLOAD_CID, WORKLOAD_LIN, 1),
+                  "gemv_m4": (WORKLOAD_CID, WORKLOAD_LIN, 4), "gemm_m16": (4, 0, 16),
                   "gemm_m64": (4, 0, 64)}[a.case]
     W = inputs.workload_weight(cid, li)
-    x = inputs.workload_activations(cid, li, M)
+    x = (inputs.workload_activations(cid, li, M) if M in inputs.WORKLOADS[cid].Ms else
+         inputs.activations(M, W.shape[1], seed=M + 11))
     Wt = torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16)
     del W
     qw = wq.quantize(Wt, symmetric=inputs.WORKLOADS[cid].sym)
     del Wt
     xt = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    path = "gemm" if a.case.startswith("gemm") else "gemv"
     for _ in range(3):
-        y = wq.linear(xt, qw)
+        y = wq.linear(xt, qw, path=path)
     torch.cuda.synchronize()
     if wq.last_device_status() != 0:
         raise RuntimeError("device error")
