@@ -800,11 +800,26 @@ __global__ void __launch_bounds__(256) gemv_finish_kernel(const FinishParams f) 
   const int c_last = owner_cta(ub + f.NS - 1, f.tiles, f.G);
   griddep_wait();                    // the streaming kernel's partials are complete
   if (c_first == c_last) return;
+  // All pieces' loads are issued before the first addition (they are
+  // independent), then added in slab order: one L2 round trip per batch of
+  // kBatch pieces instead of one per piece.
+  constexpr int kBatch = 8;
   float tot = 0.0f;
-  for (int c2 = c_first; c2 <= c_last; ++c2) {
-    const long long tc = (long long)c2 * f.tiles / f.G;
-    const int sa = (int)((tc > ub ? tc : ub) - ub);
-    tot += __ldcg(f.partials + ((size_t)sa * f.MP + m) * f.Npad + n);
+  for (int c0 = c_first; c0 <= c_last; c0 += kBatch) {
+    float v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int c2 = c0 + j;
+      v[j] = 0.0f;
+      if (c2 <= c_last) {
+        const long long tc = (long long)c2 * f.tiles / f.G;
+        const int sa = (int)((tc > ub ? tc : ub) - ub);
+        v[j] = __ldcg(f.partials + ((size_t)sa * f.MP + m) * f.Npad + n);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      if (c0 + j <= c_last) tot += v[j];
   }
   f.y[(size_t)m * f.N + n] = tot;
 }
