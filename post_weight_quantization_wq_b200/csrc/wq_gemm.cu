@@ -550,16 +550,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (prev == (unsigned)(c_last - c_first)) {
               __threadfence();
               const int m_end = prm.M < m0 + EC ? prm.M : m0 + EC;
-              if (n < g.N)
-                for (int m = m0; m < m_end; ++m) {
-                  float tot = 0.0f;
+              if (n < g.N) {
+                // pieces in slab order; the loads of one piece for up to 16
+                // rows of x are independent and go out together
+                constexpr int kRB = EC < 16 ? EC : 16;
+                for (int mb = m0; mb < m_end; mb += kRB) {
+                  float tot[kRB];
+#pragma unroll
+                  for (int m = 0; m < kRB; ++m) tot[m] = 0.0f;
                   for (int c2 = c_first; c2 <= c_last; ++c2) {
                     const long long tc = (long long)c2 * prm.tiles / G;
                     const int sa = (int)((tc > ub ? tc : ub) - ub);
-                    tot += __ldcg(prm.partials + ((size_t)sa * MPAD + m) * g.Npad + n);
+                    const float* src = prm.partials + ((size_t)sa * MPAD + mb) * g.Npad + n;
+#pragma unroll
+                    for (int m = 0; m < kRB; ++m)
+                      if (mb + m < m_end) tot[m] += __ldcg(src + (size_t)m * g.Npad);
                   }
-                  prm.y[(size_t)m * g.N + n] = tot;
+#pragma unroll
+                  for (int m = 0; m < kRB; ++m)
+                    if (mb + m < m_end) prm.y[(size_t)(mb + m) * g.N + n] = tot[m];
                 }
+              }
               if (lane == 0) *ctr = 0u;
             }
           }

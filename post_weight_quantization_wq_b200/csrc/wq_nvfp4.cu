@@ -419,8 +419,19 @@ __global__ void nvfp4_finish_kernel(const float* __restrict__ partials, int KT, 
   const int c_first = (int)(((s_lo + 1) * G - 1) / T);
   const int c_last = (int)(((s_hi + 1) * G - 1) / T);
   const float* src = partials + ((size_t)b * P * MPAD + m) * 128 + (n & 127);
+  // every piece's load before the additions (in CTA order): one L2 round trip
+  // per batch of pieces
+  constexpr int kBatch = 8;
   float t = 0.0f;
-  for (int c = 0; c <= c_last - c_first; ++c) t += src[(size_t)c * MPAD * 128];
+  for (int c0 = 0; c0 <= c_last - c_first; c0 += kBatch) {
+    float v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      v[j] = c0 + j <= c_last - c_first ? src[(size_t)(c0 + j) * MPAD * 128] : 0.0f;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      if (c0 + j <= c_last - c_first) t += v[j];
+  }
   y[e] = t * (*s_w * *s_x);
 }
 
