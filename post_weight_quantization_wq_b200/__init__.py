@@ -241,9 +241,11 @@ def linear(x, qw: QuantizedWeight, inv_act_scale=None, out=None, workspace=None,
     if workspace is not None:
         _require(workspace, "workspace", torch.uint8, None, x.device)
     y = out if out is not None else torch.empty((M, qw.N), dtype=torch.float32, device=x.device)
-    # CUDA-core GEMV up to 2 rows (HBM-bound) and for the AWQ fold (its
-    # scaled activations are not exact in a bf16 tensor-core operand);
-    # tensor-core GEMM from 3 rows on, where the GEMV becomes issue-bound
+    # wq_gemv_w4a16 up to 2 rows and for the AWQ fold (its scaled activations
+    # are not exact in a bf16 tensor-core operand); wq_gemm_w4a16 from 3 rows
+    # on.  Both entries run the int8 tensor-core kernel where it applies
+    # (K a multiple of 512: M = 2..8 / M <= 16); otherwise the bf16 skinny
+    # GEMM beats the CUDA-core GEMV from about M = 3.
     if path is None:
         path = "gemv" if (M <= GEMV_MAX_ROWS or inv_act_scale is not None) else "gemm"
     if workspace is None:

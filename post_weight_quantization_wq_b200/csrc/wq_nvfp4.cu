@@ -148,6 +148,101 @@ __global__ void nvfp4_finish_scale_kernel(unsigned* amax_bits) {
   *reinterpret_cast<float*>(amax_bits) = __fdiv_rn(fmaxf(amax, 1e-8f), 2688.0f);
 }
 
+// ---- activations of the W4A4 linear: the same quantizer in two kernels
+// with no memset, launched as programmatic dependents so that the FP4 GEMM
+// behind them can start loading weights while x is quantized.
+constexpr int kActAmaxCtas = 148;            // CTAs of the amax pass (at most)
+
+// Per-CTA largest finite |x| into partial[blockIdx.x] (non-finite values are
+// left out, as in the tensor quantizer).
+__global__ void __launch_bounds__(256) nvfp4_act_amax_kernel(const uint16_t* __restrict__ A,
+                                                             long long n,
+                                                             float* __restrict__ partial) {
+  griddep_launch_dependents();
+  griddep_wait();                              // x may come from the previous kernel
+  __shared__ float red[8];
+  float m = 0.0f;
+  const long long n8 = n / 8;                  // n is a multiple of 16
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+       i += (long long)gridDim.x * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(A)[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = fabsf(__uint_as_float(w[q] << 16));
+      const float b = fabsf(__uint_as_float(w[q] & 0xFFFF0000u));
+      if (a <= 3.402823466e38f) m = fmaxf(m, a);
+      if (b <= 3.402823466e38f) m = fmaxf(m, b);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = red[0];
+    for (int w = 1; w < 8; ++w) t = fmaxf(t, red[w]);
+    partial[blockIdx.x] = t;
+  }
+}
+
+// Every CTA reduces the partial maxima to S (reading F3; CTA 0 stores it),
+// then quantizes as nvfp4_quantize_kernel does with the block scales in the
+// tensor-core layout, and writes zero scales for the padding rows [R, RP)
+// of the activation tile (finite, so that 0-coded padding rows stay 0).
+__global__ void __launch_bounds__(256) nvfp4_act_quantize_kernel(
+    const uint16_t* __restrict__ A, int R, int RP, int C, const float* __restrict__ partial,
+    int np, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, float* __restrict__ s_out) {
+  griddep_launch_dependents();
+  griddep_wait();                              // the partial maxima are complete
+  __shared__ float red[8];
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) m = fmaxf(m, partial[i]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float amax = red[0];
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  const float S = __fdiv_rn(fmaxf(amax, 1e-8f), 2688.0f);     // 6 * 448
+  const float S6 = __fmul_rn(6.0f, S);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *s_out = S;
+  const int CB = C / kFp4Block;
+  const long long nblk = (long long)R * CB;
+  const long long npad = (long long)(RP - R) * CB;
+  for (long long bi = blockIdx.x * (long long)blockDim.x + threadIdx.x; bi < nblk + npad;
+       bi += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(bi / CB), cb = (int)(bi % CB);
+    uint32_t sb = 0;
+    if (bi < nblk) {
+      const uint4* src = reinterpret_cast<const uint4*>(A + (size_t)r * C + (size_t)cb * kFp4Block);
+      const uint4 u0 = src[0], u1 = src[1];
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float v[16];
+      float am = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        am = fmaxf(am, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
+      }
+      sb = e4m3_encode(__fdiv_rn(am, S6));
+      if (sb == 0) sb = 1;
+      const float eff = __fmul_rn(e4m3_decode(sb), S);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        lo |= e2m1_encode(__fdiv_rn(v[i], eff)) << (4 * i);
+        hi |= e2m1_encode(__fdiv_rn(v[8 + i], eff)) << (4 * i);
+      }
+      reinterpret_cast<uint2*>(codes)[bi] = make_uint2(lo, hi);
+    }
+    const int t = r >> 7, m1 = (r >> 5) & 3, m0 = r & 31;
+    const int kb = cb >> 2, ks = cb & 3;
+    scales[((size_t)t * (C / 64) + kb) * 512 + m0 * 16 + m1 * 4 + ks] = (uint8_t)sb;
+  }
+}
+
 // Canonical block scales [N][K/16] -> the tensor-core scale layout.
 __global__ void nvfp4_sf_relayout_kernel(const uint8_t* __restrict__ sf, int N, int K,
                                          uint8_t* __restrict__ out) {
@@ -289,9 +384,46 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Weights never come from an earlier kernel of the stream: the first S
+    // stages' weight codes and scales are requested before waiting for the
+    // kernel that quantizes the activations, their activation parts after.
+    auto issue = [&](int st, int b, int sg, bool wpart, bool xpart) {
+      const int kb0 = 4 * sg;
+      const int nkb = KB - kb0 < 4 ? KB - kb0 : 4;
+      if (elect_one()) {
+        uint8_t* sa = smem + st * SM::kStage;
+        const uint32_t sfb = (uint32_t)nkb * 512u;
+        if (wpart) {
+          mbar_arrive_expect_tx(&full[st], (uint32_t)(SM::kA + SM::kB) + 2u * sfb);
+          tma_load_2d(sa, &wmap, sg * 128, b * 128, &full[st]);
+          bulk_copy_g2s(sa + SM::kA + SM::kB, p.w_sf + ((size_t)b * KB + kb0) * 512, sfb,
+                        &full[st]);
+        }
+        if (xpart) {
+          tma_load_2d(sa + SM::kA, &xmap, sg * 128, 0, &full[st]);
+          bulk_copy_g2s(sa + SM::kA + SM::kB + SM::kSF, p.x_sf + (size_t)kb0 * 512, sfb,
+                        &full[st]);
+        }
+      }
+      __syncwarp();
+    };
+    int npre = 0;
+    {
+      int b = b_first, s0 = 0, s1 = 0;
+      if (b < b_end) piece(b, s0, s1);
+      for (int sg = s0; npre < S && b < b_end; ++npre) {
+        issue(npre, b, sg, true, false);
+        if (++sg == s1 && ++b < b_end) {
+          piece(b, s0, s1);
+          sg = s0;
+        }
+      }
+    }
+    griddep_wait();                         // the activations' codes and scales are complete
     int i = 0;                              // stages issued by this CTA
     bool ok = true;
     for (int b = b_first; b < b_end && ok; ++b) {
@@ -299,22 +431,13 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
       piece(b, s0, s1);
       for (int sg = s0; sg < s1; ++sg, ++i) {
         const int st = i % S;
-        if (i >= S) ok = warp_wait(&empty[st], ((i / S) - 1) & 1, p.wait_ns);
-        if (!ok) break;
-        const int kb0 = 4 * sg;
-        const int nkb = KB - kb0 < 4 ? KB - kb0 : 4;
-        if (elect_one()) {
-          uint8_t* sa = smem + st * SM::kStage;
-          const uint32_t sfb = (uint32_t)nkb * 512u;
-          mbar_arrive_expect_tx(&full[st], (uint32_t)(SM::kA + SM::kB) + 2u * sfb);
-          tma_load_2d(sa, &wmap, sg * 128, b * 128, &full[st]);
-          tma_load_2d(sa + SM::kA, &xmap, sg * 128, 0, &full[st]);
-          bulk_copy_g2s(sa + SM::kA + SM::kB, p.w_sf + ((size_t)b * KB + kb0) * 512, sfb,
-                        &full[st]);
-          bulk_copy_g2s(sa + SM::kA + SM::kB + SM::kSF, p.x_sf + (size_t)kb0 * 512, sfb,
-                        &full[st]);
+        if (i < npre) {
+          issue(st, b, sg, false, true);
+          continue;
         }
-        __syncwarp();
+        ok = warp_wait(&empty[st], ((i / S) - 1) & 1, p.wait_ns);
+        if (!ok) break;
+        issue(st, b, sg, true, true);
       }
     }
     if (!ok) {
@@ -367,6 +490,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // tensor-memory lane quadrant of this warp
+    griddep_wait();                          // the partial sums may still be read by an earlier kernel
     int lu = 0;
     for (int b = b_first; b < b_end; ++b, ++lu) {
       const int db = lu & 1;
@@ -410,6 +534,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
 __global__ void nvfp4_finish_kernel(const float* __restrict__ partials, int KT, int G, int P,
                                     int MPAD, int M, int N, const float* __restrict__ s_w,
                                     const float* __restrict__ s_x, float* __restrict__ y) {
+  griddep_launch_dependents();
+  griddep_wait();                      // the GEMM's partial sums are complete
   const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (e >= (long long)M * N) return;
   const int m = (int)(e / N), n = (int)(e % N);
@@ -466,7 +592,7 @@ size_t nvfp4_linear_workspace_bytes(int M, int N, int K) {
   const int KT = (K + kFp4StageK - 1) / kFp4StageK;
   const Fp4Split sp = fp4_split(NBt, KT);
   auto a256 = [](size_t v) { return (v + 255) / 256 * 256; };
-  return a256((size_t)M * K / 2) + a256((size_t)(K / 64) * 512) + a256(16) +
+  return a256((size_t)M * K / 2) + a256((size_t)(K / 64) * 512) + a256(16 + 4 * kActAmaxCtas) +
          a256((size_t)NBt * sp.P * fp4_mpad(M) * 128 * 4);
 }
 
@@ -505,7 +631,7 @@ static cudaError_t launch_fp4_gemm(const Fp4GemmParams& prm, const uint8_t* w_co
   if (e != cudaSuccess) return e;
   Fp4GemmParams pp = prm;
   void* args[] = {&pp, &wmap, &xmap};
-  return cudaLaunchKernel(fn, dim3((unsigned)prm.G), dim3(kFp4Threads), args, SM::kAlloc, stream);
+  return launch_pdl(fn, dim3((unsigned)prm.G), dim3(kFp4Threads), args, SM::kAlloc, stream);
 }
 
 cudaError_t launch_nvfp4_linear(const void* x, const uint8_t* packed, const float* w_scale, int M,
@@ -518,10 +644,35 @@ cudaError_t launch_nvfp4_linear(const void* x, const uint8_t* packed, const floa
   uint8_t* x_codes = ws;
   uint8_t* x_sf = x_codes + a256((size_t)M * K / 2);
   float* s_x = reinterpret_cast<float*>(x_sf + a256((size_t)(K / 64) * 512));
-  float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_x) + 256);
-  // the activations in NVFP4, their block scales in the tensor-core layout
-  cudaError_t e = launch_nvfp4_quantize(x, M, K, x_codes, x_sf, s_x, nullptr, 1, num_sms, stream);
-  if (e != cudaSuccess) return e;
+  float* amax_part = s_x + 4;
+  float* partials =
+      reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_x) + a256(16 + 4 * kActAmaxCtas));
+  // the activations in NVFP4 (their block scales in the tensor-core layout):
+  // per-CTA maxima, then the quantizer; each a programmatic dependent of the
+  // kernel before it
+  cudaError_t e;
+  {
+    const uint16_t* xp = static_cast<const uint16_t*>(x);
+    long long n = (long long)M * K;
+    long long ga = (n / 8 + 255) / 256;
+    if (ga > kActAmaxCtas) ga = kActAmaxCtas;
+    void* args[] = {&xp, &n, &amax_part};
+    if ((e = launch_pdl(reinterpret_cast<const void*>(&nvfp4_act_amax_kernel), dim3((unsigned)ga),
+                        dim3(256), args, 0, stream)) != cudaSuccess)
+      return e;
+    int R = M, RP = fp4_mpad(M), C = K, np = (int)ga;
+    const long long work = (long long)RP * (K / kFp4Block);
+    long long gq = (work + 255) / 256;
+    if (gq > (long long)num_sms * 4) gq = (long long)num_sms * 4;
+    uint8_t* codes = x_codes;
+    uint8_t* scales = x_sf;
+    const float* partp = amax_part;
+    float* sout = s_x;
+    void* qargs[] = {&xp, &R, &RP, &C, &partp, &np, &codes, &scales, &sout};
+    if ((e = launch_pdl(reinterpret_cast<const void*>(&nvfp4_act_quantize_kernel),
+                        dim3((unsigned)gq), dim3(256), qargs, 0, stream)) != cudaSuccess)
+      return e;
+  }
   Fp4GemmParams prm;
   prm.w_sf = packed + (size_t)N * K / 2;
   prm.x_sf = x_sf;
@@ -544,9 +695,13 @@ cudaError_t launch_nvfp4_linear(const void* x, const uint8_t* packed, const floa
   }
   if (e != cudaSuccess) return e;
   const long long outs = (long long)M * N;
-  nvfp4_finish_kernel<<<(unsigned)((outs + 255) / 256), 256, 0, stream>>>(
-      partials, KT, prm.G, prm.P, fp4_mpad(M), M, N, w_scale, s_x, y);
-  return cudaGetLastError();
+  const float* pp = partials;
+  int KTv = KT, Gv = prm.G, Pv = prm.P, MPv = fp4_mpad(M), Mv = M, Nv = N;
+  const float* swp = w_scale;
+  const float* sxp = s_x;
+  void* fargs[] = {&pp, &KTv, &Gv, &Pv, &MPv, &Mv, &Nv, &swp, &sxp, &y};
+  return launch_pdl(reinterpret_cast<const void*>(&nvfp4_finish_kernel),
+                    dim3((unsigned)((outs + 255) / 256)), dim3(256), fargs, 0, stream);
 }
 
 cudaError_t launch_nvfp4_quantize(const void* A, int R, int C, uint8_t* codes, uint8_t* scales,
