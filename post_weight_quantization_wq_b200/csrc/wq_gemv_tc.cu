@@ -32,8 +32,11 @@
 //   D[2m] = sum q h,  D[2m+1] = sum q l',  D[2Mp] = sum q,
 // so that exactly (l = l' + 128)
 //   sum_{k in c} q x_i = 256 D[2m] + D[2m+1] + 128 D[2Mp]
-// (every term fits in int32: 64 products of at most 15 * 128).  The chunk's
-// contribution to y is then s16 * (that - z * sum_{k in c} x_i) * 2^-e in fp32.
+// (every term fits in int32: 64 products of at most 15 * 128).  With
+// u_c = 2^-e of chunk c and the group's P = sum_{c in group} u_c * sum_{k in c} x_i
+// (the same for every weight row, prepared with the activation rows), a
+// group of two chunks adds s16 * (sum_c u_c * t_c - z * P) to y in fp32
+// (u_c * t_c is exact: u_c is a power of two).
 //
 // The planes depend on the slab of x only, not on the row tile, so a first
 // small kernel prepares them once per slab into the workspace (already in
@@ -130,7 +133,7 @@ struct TgSmem {
 struct TgParams {
   const uint8_t* packed;
   const uint8_t* planes;   // prepared B rows: [NS][4 K-blocks][2 MP rows][128 B]
-  const float2* xinfo;     // [NS][MP][8 chunks] (sum x_i, 2^-e)
+  const float2* xinfo;     // [NS][MP][8 chunks] (2^-e of the chunk, P of its group)
   float* y;                // fp32 [M][N]
   float* partials;         // fp32 [NS][MP][Npad]
   int* err;
@@ -194,8 +197,8 @@ __host__ __device__ constexpr int tg_slab_plane_bytes(int MP) { return 4 * 2 * M
 
 // One warp per (slab s, row m < MP of x): the fixed-point bytes of row m of
 // the slab (of x' = x * inv_s when inv_s is given), in the shared-memory
-// order of rows 2m and 2m + 1 of each K-block, and the chunk factors
-// (sum x_i, 2^-e).  Rows m >= M are zeros.
+// order of rows 2m and 2m + 1 of each K-block, and per chunk (2^-e, P of its
+// group of two chunks).  Rows m >= M are zeros.
 // planes: [NS][4 K-blocks][2 MP rows][128 B]; xinfo: [NS][MP][8].
 __global__ void __launch_bounds__(32 * kTgMaxM) gemv_tc_prep_kernel(const uint16_t* __restrict__ x,
                                                                     const float* __restrict__ inv_s,
@@ -292,7 +295,12 @@ __global__ void __launch_bounds__(32 * kTgMaxM) gemv_tc_prep_kernel(const uint16
   *reinterpret_cast<uint4*>(row_at(2 * m + 1)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   sx += __shfl_xor_sync(0xFFFFFFFFu, sx, 1);
   sx += __shfl_xor_sync(0xFFFFFFFFu, sx, 2);
-  if (sub == 0) xinfo[((size_t)s * MP + m) * 8 + c] = make_float2((float)sx, unscale);
+  // u * sum x_i is exact (|sum x_i| < 2^21, u a power of two); P adds the
+  // group's two chunks (lane ^ 4 holds the other one), the same sum on both
+  const float v = __fmul_rn(unscale, (float)sx);
+  const float other = __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+  const float P = (c & 1) ? __fadd_rn(other, v) : __fadd_rn(v, other);
+  if (sub == 0) xinfo[((size_t)s * MP + m) * 8 + c] = make_float2(unscale, P);
 }
 
 template <int MP>
@@ -590,27 +598,36 @@ __global__ void __launch_bounds__(kTgThreads, 1)
           }
         }
         const float2* xinfo = reinterpret_cast<const float2*>(smem + SM::kXinfo + xs * SH::kXinfo);
-        // the four chunks' accumulators, kCS at a time (bounded registers)
+        // per group of two chunks: acc = sum_c u_c t_c, then
+        // run += s16 (acc - z P); the accumulators kCS chunks at a time
         constexpr int kCS = NB >= 32 ? 1 : 2;
         const uint32_t dbase = lane_base + jd * SH::kDCols;
 #pragma unroll
-        for (int c2 = 0; c2 < 4; c2 += kCS) {
-          int dv[kCS][NB];
+        for (int gg = 0; gg < 2; ++gg) {
+          float acc[MP];
 #pragma unroll
-          for (int c1 = 0; c1 < kCS; ++c1) tmem_ld_cols<NB>(dbase + (c2 + c1) * NB, dv[c1]);
-          tmem_wait_ld();
+          for (int m = 0; m < MP; ++m) acc[m] = 0.0f;
 #pragma unroll
-          for (int c1 = 0; c1 < kCS; ++c1) {
-            const int cc = c2 + c1;
-            const int* D = dv[c1];
-            const int ones = 128 * D[2 * MP];
+          for (int c2 = 2 * gg; c2 < 2 * gg + 2; c2 += kCS) {
+            int dv[kCS][NB];
 #pragma unroll
-            for (int m = 0; m < MP; ++m) {
-              const float2 xi = xinfo[m * 8 + 4 * eh + cc];   // (sum x_i, 2^-e)
-              const int t = 256 * D[2 * m] + D[2 * m + 1] + ones;
-              run[m] += (sc[cc >> 1] * ((float)t - zc[cc >> 1] * xi.x)) * xi.y;
+            for (int c1 = 0; c1 < kCS; ++c1) tmem_ld_cols<NB>(dbase + (c2 + c1) * NB, dv[c1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c1 = 0; c1 < kCS; ++c1) {
+              const int cc = c2 + c1;
+              const int* D = dv[c1];
+              const int ones = 128 * D[2 * MP];
+#pragma unroll
+              for (int m = 0; m < MP; ++m) {
+                const int t = 256 * D[2 * m] + D[2 * m + 1] + ones;
+                acc[m] = fmaf(xinfo[m * 8 + 4 * eh + cc].x, (float)t, acc[m]);
+              }
             }
           }
+#pragma unroll
+          for (int m = 0; m < MP; ++m)
+            run[m] = fmaf(sc[gg], fmaf(-zc[gg], xinfo[m * 8 + 4 * eh + 2 * gg].y, acc[m]), run[m]);
         }
         tc_fence_before();
         __syncwarp();
