@@ -56,7 +56,8 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the offline and other-M legs")
-    ap.add_argument("--case", choices=["gemv_m1", "gemv_m4", "gemm_m16", "gemm_m64"], default=None,
+    ap.add_argument("--case", choices=["gemv_m1", "gemv_m4", "gemm_m16", "gemm_m64", "gemm_m512",
+                                       "nvfp4_m1", "nvfp4_m128"], default=None,
                     help="run one small profiling case (3 launches) and exit")
     return ap.parse_args()
 
@@ -498,7 +499,8 @@ def time_layer_awq(dev, stream):
     """The AWQ workload: the seven linears of a Llama-70B GQA decoder layer
     (q, k, v, o, gate, up, down; 455 MB packed, more than L2) quantized with
     the AWQ scale folded in, run in order through wq_gemv_w4a16 with the
-    activation factor 1/s, as one CUDA graph; M = 1 and 4."""
+    activation factor 1/s, as one CUDA graph; M = 1 and 4.  Also each linear
+    alone, over rotating copies of its weight (> 3 x L2)."""
     import numpy as np
     import torch
     import post_weight_quantization_wq_b200 as wq
@@ -555,8 +557,35 @@ def time_layer_awq(dev, stream):
             e1.record(stream)
         e1.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / (10 * reps)
+        # each linear alone: back-to-back launches over enough copies of its
+        # packed weight to exceed L2 three times
+        per = {}
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        for lin, qw, inv, xt, y, ws, wsb in runs:
+            ncopies = max(3, math.ceil(3 * l2 / qw.packed.numel()))
+            copies = [qw.packed] + [qw.packed.clone() for _ in range(ncopies - 1)]
+
+            def one(i, s_):
+                st = abi.wq_gemv_w4a16(xt, inv, copies[i % ncopies], M, lin.N, lin.K, 128, wl.sym,
+                                       1, y, ws, wsb, s_)
+                assert st == 0
+
+            steps = 20 * ncopies
+            gl = build_graphs(one, stream, steps, steps, dev)
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                gl[0].replay()
+                f0.record(stream)
+                for _ in range(3):
+                    gl[0].replay()
+                f1.record(stream)
+            f1.synchronize()
+            per[lin.name] = round(f0.elapsed_time(f1) * 1e3 / (3 * steps), 2)
+            del copies, gl
         out[f"m{M}"] = {"us_per_layer": round(us, 2), "bytes": nbytes,
-                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "launches": 7}
+                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "launches": 7,
+                        "us_per_linear_alone": per}
     if abi.wq_last_device_status(stream) != 0:
         raise RuntimeError("device error in the AWQ layer leg")
     del lins
@@ -805,7 +834,9 @@ def cpu_baseline(W, x, N, K, sym, target_s: float = 10.0):
     oracle.linear(x, P, s, z, K, sym=sym)
     per_row = (time.perf_counter() - t) / rows0
     R = int(min(N, max(rows0, target_s / max(per_row, 1e-9))))
+    tq = time.perf_counter()
     q, s, z, _ = oracle.quantize_bf16(W[:R], None, sym=sym)
+    quant_single = (time.perf_counter() - tq) / R * N * 1e6
     P = oracle.pack_u4(q, sym)
     del q
     t = time.perf_counter()
@@ -825,6 +856,7 @@ def cpu_baseline(W, x, N, K, sym, target_s: float = 10.0):
                       f"dequantize + dot per row) on {cores} threads ({el_mt:.2f} s) and on one "
                       f"thread ({el:.1f} s), scaled to the full linear",
             "single_thread_value": round(single, 1),
+            "quantize_single_thread_us": round(quant_single, 1),
             "host_cpu": _cpu_model(), "host_cores_available": os.cpu_count()}
 
 
@@ -908,16 +940,34 @@ def max_over_ranks(v, world, dev):
 def run_case(a):
     """A few launches of one kernel on one workload, for profilers: gemv_m1 /
     gemv_m4 = wq_gemv_w4a16 on 8192x28672 at M = 1 (CUDA cores) / 4 (int8
-    tensor cores); gemm_m16 / gemm_m64 = wq_gemm_w4a16 on 28672x8192 at
-    M = 16 (int8 tensor cores) / 64 (bf16 tensor cores), asymmetric.  About
+    tensor cores); gemm_m16 / gemm_m64 / gemm_m512 = wq_gemm_w4a16 on
+    28672x8192 at M = 16 (int8 tensor cores) / 64 (bf16 skinny kernel) / 512
+    (many-row prefill kernel), asymmetric; nvfp4_m1 / nvfp4_m128 =
+    wq_nvfp4_linear on 8192x28672 at M = 1 / 28672x8192 at M = 128.  About
     1 GB on the device."""
     import numpy as np
     import torch
     import post_weight_quantization_wq_b200 as wq
     from post_weight_quantization_wq_b200 import inputs
+    if a.case.startswith("nvfp4"):
+        cid, li, M = {"nvfp4_m1": (WORKLOAD_CID, WORKLOAD_LIN, 1), "nvfp4_m128": (4, 0, 128)}[a.case]
+        W = inputs.workload_weight(cid, li)
+        Wt = torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16)
+        x = inputs.activations(M, W.shape[1], seed=M + 11)
+        del W
+        qw = wq.nvfp4_quantize(Wt)
+        del Wt
+        xt = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+        for _ in range(3):
+            y = wq.nvfp4_linear(xt, qw)
+        torch.cuda.synchronize()
+        if wq.last_device_status() != 0:
+            raise RuntimeError("device error")
+        print(json.dumps({"case": a.case, "y_sum": float(y.double().sum())}))
+        return
     cid, li, M = {"gemv_m1": (WORKLOAD_CID, WORKLOAD_LIN, 1),
                   "gemv_m4": (WORKLOAD_CID, WORKLOAD_LIN, 4), "gemm_m16": (4, 0, 16),
-                  "gemm_m64": (4, 0, 64)}[a.case]
+                  "gemm_m64": (4, 0, 64), "gemm_m512": (4, 0, 512)}[a.case]
     W = inputs.workload_weight(cid, li)
     x = (inputs.workload_activations(cid, li, M) if M in inputs.WORKLOADS[cid].Ms else
          inputs.activations(M, W.shape[1], seed=M + 11))
