@@ -44,8 +44,8 @@ START_DELAY_CYCLES = 500_000                # ~0.25 ms of SM clock ahead of the 
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": "20ec021dcbfc87a64136d3d22a0aa071f1261b34335a297d582377226c1d48e6",
-               "bytes_per_launch": 124880896 + 4332288}
+NCU_TRAFFIC = {"sources_sha256": "cee50bff8ffafd59bb2749635eabc5c6dea8412bfbff4955913041887afa5a6f",
+               "bytes_per_launch": 124883456 + 3779328}
 
 
 def _args():

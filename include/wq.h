@@ -171,8 +171,8 @@ size_t wq_gemm_workspace_bytes(int M, int N, int K);
  * u[m][k] = fp32(x[m][k]) * inv_act_scale[k] (the AWQ fold, inv_act_scale =
  * 1/s, one rounded fp32 product).
  *   - The integer paths: M = 2..8 with K a multiple of 512 (int8 tensor
- *     cores, tcgen05.mma kind::i8, with or without inv_act_scale), and
- *     M <= 4 without inv_act_scale otherwise (CUDA cores, dp4a).  Each
+ *     cores, tcgen05.mma kind::i8), and M <= 4 otherwise (CUDA cores,
+ *     dp4a), both with or without inv_act_scale.  Each
  *     64-input chunk of a row of u is rounded to 16-bit fixed point,
  *     x' = rn(u * 2^e) * 2^-e with e chosen so that the chunk's largest |u|
  *     lies in [2^14, 2^15) (a bf16 value there, and any value with at most
@@ -183,9 +183,8 @@ size_t wq_gemm_workspace_bytes(int M, int N, int K);
  *     holding a NaN or an infinity makes every output of its row NaN.  Both
  *     integer kernels give the same per-chunk integers and differ only in
  *     the order of the fp32 additions of the chunks' contributions.
- *   - otherwise (M = 1 with inv_act_scale, or K not a multiple of 512 with
- *     M = 5..8 or with inv_act_scale) x' = u, multiplied in fp32 on the
- *     CUDA cores.
+ *   - otherwise (M = 5..8 with K not a multiple of 512) x' = u, multiplied
+ *     in fp32 on the CUDA cores.
  *   x        bf16 [M][K];      inv_act_scale fp32 [K] or NULL;
  *   packed   the weight in kernel layout `layout` (from wq_pack_layout);
  *   y        fp32 [M][N] out;

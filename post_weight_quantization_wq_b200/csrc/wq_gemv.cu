@@ -202,7 +202,7 @@ __device__ __forceinline__ int owner_cta(long long u, long long T, int G) {
 template <int MP, bool IDOT>
 struct XSlice {
   uint4 xb[MP][2];
-  float4 inv[IDOT ? 1 : 4];
+  float4 inv[4];
 };
 
 // Read lane l's share (inputs 16l .. 16l+15 of the slab) from a raw slot.
@@ -231,7 +231,21 @@ __device__ __forceinline__ void read_x_slice(XSlice<MP, IDOT>& xs, const uint8_t
   }
 }
 
+// Integer path with the AWQ factor: lane l's 16 factors of slab s, read from
+// global memory (the factor is small and stays in L2); issued before the
+// producer's waits so that their latency overlaps them.
 template <int MP, bool IDOT>
+__device__ __forceinline__ void load_inv_slice(XSlice<MP, IDOT>& xs, const GemvParams& prm, int s,
+                                               int lane) {
+  const bool ok = s * kSlabK + 16 * lane < prm.g.K;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    xs.inv[q] = (ok && prm.inv_s)
+                    ? __ldg(reinterpret_cast<const float4*>(prm.inv_s + (size_t)s * kSlabK + 16 * lane) + q)
+                    : make_float4(1.f, 1.f, 1.f, 1.f);
+}
+
+template <int MP, bool IDOT, bool AWQI>
 __device__ __forceinline__ void store_x_slice(const XSlice<MP, IDOT>& xs, uint8_t* stage,
                                               const GemvParams& prm, int lane) {
   using SL = StageLayout<MP, IDOT>;
@@ -247,15 +261,29 @@ __device__ __forceinline__ void store_x_slice(const XSlice<MP, IDOT>& xs, uint8_
       // there: bf16 has 8 significant bits), every other value within half a
       // step 2^-e.  x_i = 256 h + l is stored as signed high bytes h and
       // unsigned low bytes l, ordered like the code bytes of an interleaved
-      // word (see dp4a_word).  A chunk holding a NaN or an infinity stores
-      // zeros and a NaN factor, so the rows it meets come out NaN.
+      // word (see dp4a_word).  With the AWQ factor the chunk holds
+      // u = fp32(x) * inv (one rounding) instead of x.  A chunk holding a NaN
+      // or an infinity stores zeros and a NaN factor, so the rows it meets
+      // come out NaN.
       float xf[16];
       bool bad = false;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         xf[2 * q] = bf16_lo(r[q]);
         xf[2 * q + 1] = bf16_hi(r[q]);
-        bad |= (r[q] & 0x7F80u) == 0x7F80u || (r[q] & 0x7F800000u) == 0x7F800000u;
+        if constexpr (!AWQI)
+          bad |= (r[q] & 0x7F80u) == 0x7F80u || (r[q] & 0x7F800000u) == 0x7F800000u;
+      }
+      if constexpr (AWQI) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          xf[4 * q] = __fmul_rn(xf[4 * q], xs.inv[q].x);
+          xf[4 * q + 1] = __fmul_rn(xf[4 * q + 1], xs.inv[q].y);
+          xf[4 * q + 2] = __fmul_rn(xf[4 * q + 2], xs.inv[q].z);
+          xf[4 * q + 3] = __fmul_rn(xf[4 * q + 3], xs.inv[q].w);
+        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q) bad |= !(fabsf(xf[q]) <= 3.402823466e38f);   // NaN or infinity
       }
       float amax = 0.0f;
 #pragma unroll
@@ -381,7 +409,7 @@ __host__ __device__ constexpr size_t gemv_team_smem() {
 // so more of the shared memory is in flight (EARLY; it needs registers for
 // all of the lane's codes, so it is used where a lane covers one pass of
 // rows; otherwise the stage is released after the arithmetic).
-template <int MP, int JQ, int STAGES, int XR, int RAWS, int VC, bool IDOT, bool EARLY>
+template <int MP, int JQ, int STAGES, int XR, int RAWS, int VC, bool IDOT, bool EARLY, bool AWQI>
 __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvParams prm) {
   using SL = StageLayout<MP, IDOT>;
   extern __shared__ __align__(128) uint8_t smem_all[];
@@ -478,7 +506,8 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
     auto issue_raw = [&](int slot, int slab) {       // lane 0 only
       uint8_t* dst = raw_ring + slot * SL::kRawBytes;
       const int gsx = slab_groups(g, slab);
-      const uint32_t xb = gsx * kGroup * 2, ib = prm.inv_s ? gsx * kGroup * 4 : 0;
+      // the integer path reads its AWQ factors from global memory instead
+      const uint32_t xb = gsx * kGroup * 2, ib = (prm.inv_s && !IDOT) ? gsx * kGroup * 4 : 0;
       mbar_arrive_expect_tx(&raw_bar[slot], prm.M * xb + ib);
       for (int m = 0; m < prm.M; ++m)
         bulk_copy_g2s(dst + m * kSlabK * 2, prm.x + (size_t)m * g.K + slab * kSlabK, xb,
@@ -496,6 +525,8 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
     for (int i = 0; i < ntiles; ++i) {
       const int xs = i % XR;
       const int rs = i % RAWS;
+      XSlice<MP, IDOT> xsl;
+      if constexpr (AWQI) load_inv_slice<MP, IDOT>(xsl, prm, ps, lane);
       bool ok = true;
       if (i >= XR) ok = mbar_wait_bounded(&xempty_bar[xs], ((i / XR) - 1) & 1, prm.wait_ns);
       ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
@@ -510,9 +541,8 @@ __global__ void __launch_bounds__(kGemvThreads * VC, 1) gemv_w4a16_kernel(GemvPa
         }
         break;
       }
-      XSlice<MP, IDOT> xsl;
       read_x_slice<MP, IDOT>(xsl, raw_ring + rs * SL::kRawBytes, prm, ps, lane);
-      store_x_slice<MP, IDOT>(xsl, x_ring + xs * SL::kXSlot, prm, lane);
+      store_x_slice<MP, IDOT, AWQI>(xsl, x_ring + xs * SL::kXSlot, prm, lane);
       mbar_arrive(&xfull_bar[xs]);
       ps = next_slab(ps);
       __syncwarp();                      // every lane has read raw slot rs
@@ -832,11 +862,12 @@ struct GemvConfig {
   int teams;               // virtual CTAs per CTA
 };
 
-template <int MP, int JQ, int STAGES, int XR, int RAWS, int VC, bool IDOT, bool EARLY>
+template <int MP, int JQ, int STAGES, int XR, int RAWS, int VC, bool IDOT, bool EARLY,
+          bool AWQI = false>
 static GemvConfig gemv_config() {
   GemvConfig c;
   c.fn = reinterpret_cast<const void*>(
-      &gemv_w4a16_kernel<MP, JQ, STAGES, XR, RAWS, VC, IDOT, EARLY>);
+      &gemv_w4a16_kernel<MP, JQ, STAGES, XR, RAWS, VC, IDOT, EARLY, AWQI>);
   c.smem = VC * gemv_team_smem<MP, STAGES, XR, RAWS, IDOT>();
   c.teams = VC;
   return c;
@@ -844,18 +875,18 @@ static GemvConfig gemv_config() {
 
 static int padded_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
-// Integer (dp4a) path for M <= 4 without an activation scale; packed fp32
-// path for the AWQ fold and for M > 4 (where one widening per code is shared
-// by 8 rows).  Teams x (weight stages, activation slots, raw slots) fill the
+// Integer (dp4a) path for M <= 4, with or without the AWQ factor (applied
+// in fp32 before the fixed point); packed fp32 path for M > 4 (where one
+// widening per code is shared by 8 rows).  Teams x (weight stages, activation slots, raw slots) fill the
 // shared memory of one CTA per SM; two teams keep the registers for a tile's
 // codes held between the stage release and the arithmetic.
 static GemvConfig pick_gemv(int M, bool awq) {
   switch (padded_m(M)) {
-    case 1: return awq ? gemv_config<1, 4, 3, 2, 2, 2, false, true>()
+    case 1: return awq ? gemv_config<1, 2, 3, 3, 2, 2, true, true, true>()
                        : gemv_config<1, 2, 3, 3, 2, 2, true, true>();
-    case 2: return awq ? gemv_config<2, 2, 5, 2, 2, 1, false, false>()
+    case 2: return awq ? gemv_config<2, 2, 3, 2, 3, 2, true, false, true>()
                        : gemv_config<2, 2, 3, 2, 3, 2, true, false>();
-    case 4: return awq ? gemv_config<4, 2, 5, 2, 2, 1, false, false>()
+    case 4: return awq ? gemv_config<4, 2, 5, 2, 3, 1, true, false, true>()
                        : gemv_config<4, 2, 5, 2, 3, 1, true, false>();
     default: return gemv_config<8, 2, 5, 2, 2, 1, false, false>();
   }
