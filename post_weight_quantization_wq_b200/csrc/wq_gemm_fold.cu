@@ -14,11 +14,12 @@
 //   * four dequantizing warps write the bf16 integers 128 + q (exact) into a
 //     128-byte-swizzled, K-major A tile in shared memory;
 //   * one lane issues 8 tcgen05.mma (M = 128, N = MT, K = 16, both operands
-//     from shared-memory descriptors) into one of two fp32 accumulators in
+//     from shared-memory descriptors) into one of four fp32 accumulators in
 //     tensor memory;
-//   * four fold warps add s16 * (D - (128 + z) * sum_k x) to the running sum,
-//     which also lives in tensor memory (so the registers stay small at
-//     MT = 128), then release the accumulator.
+//   * eight fold warps (two per tensor-memory lane quadrant, MT / 2 columns
+//     each) load their part of the accumulator with one wait, release it to
+//     the MMA issuer, and add s16 * (D - (128 + z) * sum_k x) to running sums
+//     held in registers.
 // The zero point and the 128 bias never enter the bf16 operands, so every
 // dequantized value is exact.  Units along K are summed by a second kernel in
 // a fixed order.
@@ -41,7 +42,9 @@ struct FoldParams {
   uint32_t lop_mask_lo, lop_bf16_128;
 };
 
-constexpr int kFoldThreads = 10 * 32;     // TMA, MMA, 4 dequant, 4 fold warps
+constexpr int kFoldThreads = 14 * 32;     // TMA, MMA, 4 dequant, 8 fold warps
+constexpr int kFoldWarps = 8;
+constexpr int kFoldAcc = 4;               // accumulators in tensor memory
 constexpr uint32_t kFoldTmemCols = 512;
 constexpr int kFoldMetaSlots = 2;
 constexpr int kFoldMetaBytes = kTileRows * kSlabGroups * 4;   // 2 KB
@@ -56,11 +59,10 @@ struct FoldSmem {
   static constexpr int kStages = MT >= 64 ? 3 : 4;
   static constexpr int kMeta = kStages * kStage;
   static constexpr int kBar = kMeta + kFoldMetaSlots * kFoldMetaBytes;
-  static constexpr int kNumBars = 3 * kStages + 4 + 2 * kFoldMetaSlots;
+  static constexpr int kNumBars = 3 * kStages + 2 * kFoldAcc + 2 * kFoldMetaSlots;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  static constexpr int kRCol = 256;                            // running sums
-  static_assert(2 * MT <= kRCol && kRCol + MT <= (int)kFoldTmemCols, "tensor memory");
+  static_assert(kFoldAcc * MT <= (int)kFoldTmemCols, "tensor memory");
 };
 
 template <int MT>
@@ -127,9 +129,9 @@ __global__ void __launch_bounds__(kFoldThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBar);   // [S] codes + x landed
   uint64_t* afull = full + S;                                       // [S] A tile written
   uint64_t* empty = afull + S;                                      // [S] MMAs done with the stage
-  uint64_t* dfull = empty + S;                                      // [2] accumulator ready
-  uint64_t* dempty = dfull + 2;                                     // [2] accumulator folded
-  uint64_t* mfull = dempty + 2;                                     // [meta] landed
+  uint64_t* dfull = empty + S;                                      // accumulator ready
+  uint64_t* dempty = dfull + kFoldAcc;                              // accumulator read
+  uint64_t* mfull = dempty + kFoldAcc;                              // [meta] landed
   uint64_t* mempty = mfull + kFoldMetaSlots;                        // [meta] read
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mempty + kFoldMetaSlots);
 
@@ -144,13 +146,13 @@ __global__ void __launch_bounds__(kFoldThreads, 1)
       mbar_init(&afull[i], 4);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kFoldAcc; ++i) {
       mbar_init(&dfull[i], 1);
-      mbar_init(&dempty[i], 4);
+      mbar_init(&dempty[i], kFoldWarps);
     }
     for (int i = 0; i < kFoldMetaSlots; ++i) {
       mbar_init(&mfull[i], 1);
-      mbar_init(&mempty[i], 4);
+      mbar_init(&mempty[i], kFoldWarps);
     }
     fence_mbarrier_init();
   }
@@ -222,10 +224,10 @@ __global__ void __launch_bounds__(kFoldThreads, 1)
     bool ok = true;
     int done = 0;
     for (int j = 0; j < ngr; ++j) {
-      const int st = j % S, db = j & 1;
+      const int st = j % S, db = j % kFoldAcc;
       ok = warp_wait(&afull[st], (j / S) & 1, p.wait_ns) &&
            warp_wait(&full[st], (j / S) & 1, p.wait_ns) &&
-           (j < 2 || warp_wait(&dempty[db], ((j / 2) - 1) & 1, p.wait_ns));
+           (j < kFoldAcc || warp_wait(&dempty[db], ((j / kFoldAcc) - 1) & 1, p.wait_ns));
       if (!ok) break;
       tc_fence_after();
       if (elect_one()) {
@@ -245,7 +247,8 @@ __global__ void __launch_bounds__(kFoldThreads, 1)
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kDevErrTimeout);
-      if (done > 0) warp_wait(&dfull[(done - 1) & 1], ((done - 1) / 2) & 1, p.drain_ns);
+      if (done > 0)
+        warp_wait(&dfull[(done - 1) % kFoldAcc], ((done - 1) / kFoldAcc) & 1, p.drain_ns);
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ dequantize
@@ -286,10 +289,14 @@ __global__ void __launch_bounds__(kFoldThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ fold
+    constexpr int EC = MT / 2;               // accumulator columns of this warp
     const int q = warp & 3;                  // tensor-memory lane quadrant
+    const int half = (warp - 6) >> 2;        // columns half * EC .. half * EC + EC - 1
     const int row = q * 32 + lane;           // row of the tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t rcol = tmem_base + lane_off + SM::kRCol;
+    float run[EC];
+#pragma unroll
+    for (int c = 0; c < EC; ++c) run[c] = 0.0f;
     float scs[kSlabGroups], czs[kSlabGroups];
     int metas = 0;
     bool ok = true;
@@ -324,55 +331,52 @@ __global__ void __launch_bounds__(kFoldThreads, 1)
 #pragma unroll
       for (int t = 1; t < kSlabGroups; ++t)
         if (gg == t) { sc = scs[t]; cz = czs[t]; }
-      const int db = j & 1;
-      ok = warp_wait(&dfull[db], (j / 2) & 1, p.wait_ns);
+      const int db = j % kFoldAcc;
+      ok = warp_wait(&dfull[db], (j / kFoldAcc) & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      const float* xs = p.xsum + (size_t)gidx * p.Mpad + u.mt * MT;
-      const uint32_t dcol = tmem_base + lane_off + db * MT;
-#pragma unroll 1
-      for (int c0 = 0; c0 < MT; c0 += 16) {
-        float d[16], rr[16];
-        tmem_ld16(dcol + c0, d);
-        if (j > 0) tmem_ld16(rcol + c0, rr);
-        tmem_wait_ld();
-        uint32_t o[16];
+      // this warp's columns of the accumulator in parts of up to 32 columns
+      // (one wait each); the accumulator goes back to the MMA issuer as soon
+      // as the last part is in registers, before its arithmetic
+      constexpr int kPart = EC < 32 ? EC : 32;
+      const uint32_t dcol = tmem_base + lane_off + db * MT + half * EC;
+      const float* xs = p.xsum + (size_t)gidx * p.Mpad + u.mt * MT + half * EC;
 #pragma unroll
-        for (int i = 0; i < 16; i += 4) {
-          const float4 x4 = __ldg(reinterpret_cast<const float4*>(xs + c0 + i));
+      for (int p0 = 0; p0 < EC; p0 += kPart) {
+        float d[kPart];
+#pragma unroll
+        for (int c0 = 0; c0 < kPart; c0 += 16) {
+          if constexpr (kPart >= 16) tmem_ld16(dcol + p0 + c0, d + c0);
+          else tmem_ld8(dcol + p0 + c0, d + c0);
+        }
+        tmem_wait_ld();
+        if (p0 + kPart == EC) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dempty[db]);
+        }
+#pragma unroll
+        for (int i = 0; i < kPart; i += 4) {
+          const float4 x4 = __ldg(reinterpret_cast<const float4*>(xs + p0 + i));
           const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float part = sc * __fmaf_rn(-cz, xv[t], d[i + t]);
-            o[i + t] = __float_as_uint(j > 0 ? rr[i + t] + part : part);
-          }
+          for (int t = 0; t < 4; ++t)
+            run[p0 + i + t] = __fmaf_rn(sc, __fmaf_rn(-cz, xv[t], d[i + t]), run[p0 + i + t]);
         }
-        tmem_st16(rcol + c0, o);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&dempty[db]);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kDevErrTimeout);
     } else if (ngr > 0) {
       // the unit's sums: y (one K split) or a partial
       const int n = u.b * kTileRows + row;
-      tc_fence_after();
-#pragma unroll 1
-      for (int c0 = 0; c0 < MT; c0 += 16) {
-        float rr[16];
-        tmem_ld16(rcol + c0, rr);
-        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int m = u.mt * MT + c0 + i;
-          if (p.KS == 1) {
-            if (m < p.M && n < g.N) p.out[(size_t)m * g.N + n] = rr[i];
-          } else if (m < p.M) {
-            p.out[((size_t)u.ks * p.Mpad + m) * g.Npad + n] = rr[i];
-          }
+      for (int i = 0; i < EC; ++i) {
+        const int m = u.mt * MT + half * EC + i;
+        if (p.KS == 1) {
+          if (m < p.M && n < g.N) p.out[(size_t)m * g.N + n] = run[i];
+        } else if (m < p.M) {
+          p.out[((size_t)u.ks * p.Mpad + m) * g.Npad + n] = run[i];
         }
       }
     }
