@@ -23,6 +23,7 @@ import argparse
 import csv
 import datetime as dt
 import hashlib
+import re
 import io
 import json
 import math
@@ -42,9 +43,10 @@ FALLBACK_HBM_GBS = 6650.0
 START_DELAY_CYCLES = 500_000                # ~0.25 ms of SM clock ahead of the start event
 
 # DRAM bytes per GEMV launch from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum) and the hash of the kernel sources it was taken on;
+# dram__bytes_write.sum) and the hash of the kernel sources (code only,
+# comments removed) it was taken on;
 # reported only while the sources are unchanged.
-NCU_TRAFFIC = {"sources_sha256": "cee50bff8ffafd59bb2749635eabc5c6dea8412bfbff4955913041887afa5a6f",
+NCU_TRAFFIC = {"sources_sha256": "10e1d16873f7fe3f44f4b7ebdefe2a62826ba7efe2948561dd2b7651b67cea0b",
                "bytes_per_launch": 124883456 + 3779328}
 
 
@@ -68,11 +70,19 @@ def algorithmic_bytes(M: int, N: int, K: int, sym: bool) -> int:
     return N * K // 2 + 2 * N * K // 128 + (0 if sym else 2 * N * K // 128) + 2 * M * K + 4 * M * N
 
 
+def _code_only(src: str) -> str:
+    """The source with comments and blank lines removed, so that the hash
+    changes with the code and not with its comments."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_sources_sha() -> str:
     h = hashlib.sha256()
     for f in ("wq_gemv.cu", "wq_common.cuh"):
-        with open(os.path.join(ROOT, "post_weight_quantization_wq_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "post_weight_quantization_wq_b200", "csrc", f)) as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()
 
 

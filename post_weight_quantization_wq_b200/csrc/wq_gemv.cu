@@ -1,5 +1,7 @@
 // wq_gemv.cu -- W4A16 decode linear for M = 1..8 activation rows on the CUDA
 // cores:  y[m][n] = sum_g s16[n][g] * sum_{k in g} x'[m][k] * (q[n][k] - z[n][g]).
+// (wq_gemv_w4a16 runs it at M = 1, and at every M whose K is not a multiple of
+// 512; the int8 tensor-core kernel of wq_gemv_tc.cu takes the other shapes.)
 //
 // Weight-only 4-bit decode is bound by the bytes of the weights ("推理优化中
 // “用精度换性能“的核心技术：量化", section 一; "3.6 量化(Quantization)",
@@ -24,14 +26,15 @@
 //   * programmatic dependent launch: the first weight tiles are requested
 //     before the kernel waits for the previous kernel of the stream;
 //   * dequantization in registers without conversion instructions.  Integer
-//     path (no activation scale, M <= 4): the producer rounds each 64-input
-//     chunk of x to integers x_i = rn(x * 2^e), e putting the chunk's largest
-//     |x| in [2^14, 2^15); two masks per code word leave the 8 codes in place
+//     path (M <= 4): the producer rounds each 64-input chunk of u = x (or
+//     u = fp32(x) * (1/s) with the AWQ factor, a separate kernel instance) to
+//     integers x_i = rn(u * 2^e), e putting the chunk's largest |u| in
+//     [2^14, 2^15); two masks per code word leave the 8 codes in place
 //     as bytes (q or 16 q), and four dp4a per word and row of x (unsigned code
 //     bytes times signed high / unsigned low activation bytes, int32
 //     accumulators) give sum q x_i exactly; each (row, chunk) sum then loses
-//     z * sum x_i and is scaled by s16 * 2^-e in fp32.  Packed path (AWQ
-//     fold, M = 8): bf16 pairs 128 + q (mask into 0x43004300) are widened to
+//     z * sum x_i and is scaled by s16 * 2^-e in fp32.  Packed path
+//     (M = 5..8): bf16 pairs 128 + q (mask into 0x43004300) are widened to
 //     the fp32 code q - z by a mixed-precision add and packed fp32x2 FMAs
 //     multiply them with the fp32 activations;
 //   * 8 lanes share a row of a tile, lane p covering inputs 64p..64p+63 of
